@@ -1,0 +1,90 @@
+"""The seeded generator reproduces the input distributions of the Kimi K3
+report's KDA layer and respects the decay bounds the report prints
+(section 2.1.1, Eq. 5): g in (g_min, 0) with g_min = -5, alpha > e^-5 ~ 6.7e-3,
+and every 16-token window of log-decay inside (-80, 0)."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_117_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_bounds():
+    vals = {}
+    for line in open(os.path.join(GOLDEN, "decay_bounds.txt")):
+        if line.strip() and not line.startswith("#"):
+            name, val = line.split()
+            vals[name] = float(val)
+    return vals
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "prefill_h16_t4k", "batched_b8_h32_t8k"])
+def test_decay_bounds(name):
+    gb = _golden_bounds()
+    w = synth.WORKLOADS[name]
+    assert synth.G_MIN == gb["g_min"]
+    heads = [0, w.H - 1] + synth.fast_decay_heads(w).tolist()
+    for h in heads:
+        x = synth.head_inputs(w, 0, h, T=512 if w.T > 512 else None)
+        g = x["g"]
+        # rounding to bf16 may land exactly on the bounds, hence closed interval
+        assert g.min() >= gb["g_min"] and g.max() <= 0.0
+        assert np.exp(g).min() >= math.exp(gb["g_min"]) >= gb["alpha_lower_bound"] - 1e-4
+        n = int(gb["tile_tokens"])
+        win = np.lib.stride_tricks.sliding_window_view(g, n, axis=0).sum(axis=-1)
+        assert win.min() >= gb["tile_cumulative_log_decay_min"]
+        # e^80 (the largest reciprocal rescale) is finite in bf16 and fp32
+        assert torch.isfinite(torch.tensor(math.exp(-gb["tile_cumulative_log_decay_min"]), dtype=torch.bfloat16))
+
+
+def test_value_distributions():
+    w = synth.WORKLOADS["prefill_h16_t4k"]
+    x = synth.head_inputs(w, 0, 3)
+    np.testing.assert_allclose(np.linalg.norm(x["q"], axis=1), 1.0, atol=4e-3)
+    np.testing.assert_allclose(np.linalg.norm(x["k"], axis=1), 1.0, atol=4e-3)
+    assert abs(x["v"].mean()) < 0.02 and abs(x["v"].std() - 1.0) < 0.02
+    assert 0.0 < x["beta"].min() and x["beta"].max() < 1.0 and abs(x["beta"].mean() - 0.5) < 0.02
+    assert abs(x["h0"].std() - 0.02) < 0.002
+    # stored values are exactly representable in bf16
+    for name in ("q", "k", "v", "g", "beta"):
+        t = torch.from_numpy(x[name])
+        assert torch.equal(t.to(torch.bfloat16).to(torch.float64), t)
+
+
+def test_fast_decay_heads_push_toward_bound():
+    w = synth.WORKLOADS["batched_b8_h32_t8k"]
+    fast = synth.fast_decay_heads(w)
+    assert len(fast) == round(0.1 * w.H) == 3
+    slow = [h for h in range(w.H) if h not in fast][0]
+    gf = synth.head_inputs(w, 0, int(fast[0]), T=256)["g"]
+    gs = synth.head_inputs(w, 0, slow, T=256)["g"]
+    # e^A ~ e^2 sharpens the sigmoid: more tokens sit near g_min
+    assert (gf < -4.5).mean() > 2 * (gs < -4.5).mean()
+
+
+def test_heads_are_reproducible_and_independent():
+    w = synth.WORKLOADS["tiny_f32"]
+    a = synth.head_inputs(w, 0, 1)
+    b = synth.head_inputs(w, 0, 1)
+    c = synth.head_inputs(w, 0, 0)
+    assert all(np.array_equal(a[n], b[n]) for n in a)
+    assert not np.array_equal(a["q"], c["q"])
+    full = synth.prefill_inputs(w)
+    assert torch.equal(full["q"][0, 1], torch.from_numpy(a["q"]).float())
+    # prefix property: a shorter draw is the prefix of the longer one
+    p = synth.head_inputs(w, 0, 1, T=20)
+    assert np.array_equal(p["q"], a["q"][:20]) and np.array_equal(p["g"], a["g"][:20])
+
+
+def test_algorithmic_counts():
+    w = synth.WORKLOADS["prefill_h16_t4k"]
+    assert synth.flops_per_token_head(128, 128, 64) == 140629.33333333334 or \
+        abs(synth.flops_per_token_head(128, 128, 64) - 140629.33) < 0.01
+    assert synth.prefill_bytes(w) == 16 * (4096 * 1282 + 2 * 65536)
+    d = synth.WORKLOADS["decode_b256_h32"]
+    assert synth.decode_bytes_per_step(d) == 256 * 32 * 132354
