@@ -1,0 +1,216 @@
+// C-ABI layer of libkda: argument validation, planning and dispatch.
+// The interface and its contract are documented in include/kda.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "kda.h"
+#include "kda_internal.cuh"
+
+namespace kda {
+
+// Status word written by kernels whose bounded waits give up or whose
+// device-side checks fail.  One per device (a __device__ variable is
+// instantiated in every context that loads the module).
+__device__ unsigned g_status_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<unsigned *> g_status_ptr[kMaxDevices];
+}  // namespace
+
+unsigned *device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned *p = g_status_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void *addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return nullptr;
+  g_status_ptr[dev].store((unsigned *)addr, std::memory_order_release);
+  return (unsigned *)addr;
+}
+
+}  // namespace kda
+
+namespace {
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void *p, size_t bytes) {
+  return Range{(uintptr_t)p, (uintptr_t)p + bytes};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+// Device must be a Blackwell datacenter part (compute capability 10.x): the
+// library is compiled for sm_100a only.
+kda_status_t check_device() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return major == 10 ? KDA_OK : KDA_ERR_UNSUPPORTED;
+}
+
+kda_status_t plan_prefill(int B, int H, int T, int dk, int dv, kda_dtype_t dtype, int chunk_size,
+                          kda_plan_t *plan) {
+  if (B < 0 || H < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  if (chunk_size != 0 && chunk_size != 16 && chunk_size != 64) return KDA_ERR_SHAPE;
+  if (chunk_size == 64) return KDA_ERR_UNSUPPORTED;  // tensor-core path not built in this version
+  kda_plan_t p;
+  p.path = KDA_PATH_SIMT16;
+  p.chunk_size = 16;
+  p.segments = 1;
+  p.launches = (B * H == 0) ? 0 : 1;
+  p.workspace = 0;
+  *plan = p;
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(kda_status_t s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_SHAPE: return "KDA_ERR_SHAPE: unsupported shape";
+    case KDA_ERR_DTYPE: return "KDA_ERR_DTYPE: unsupported dtype";
+    case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT: pointer misaligned";
+    case KDA_ERR_ALIAS: return "KDA_ERR_ALIAS: output overlaps an input";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: device or path not supported";
+    case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: device-side check failed";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+kda_status_t kda_chunk_fwd_plan(int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                int chunk_size, kda_plan_t *plan) {
+  if (!plan) return KDA_ERR_INVALID_ARG;
+  return plan_prefill(B, H, T, dk, dv, dtype, chunk_size, plan);
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                    int chunk_size) {
+  kda_plan_t p;
+  if (plan_prefill(B, H, T, dk, dv, dtype, chunk_size, &p) != KDA_OK) return (size_t)-1;
+  return p.workspace;
+}
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
+                           const void *beta, const float *h0, void *o, float *h_T, int B, int H,
+                           int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
+                           void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+  kda_plan_t plan;
+  kda_status_t st = plan_prefill(B, H, T, dk, dv, dtype, chunk_size, &plan);
+  if (st != KDA_OK) return st;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (B * H == 0) return KDA_OK;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+  const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+  const void *ptrs[] = {q, k, v, g, h0, o, h_T, workspace};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+  if (beta && ((uintptr_t)beta % e) != 0) return KDA_ERR_ALIGNMENT;
+  if (plan.workspace > 0 && (!workspace || workspace_bytes < plan.workspace)) return KDA_ERR_WORKSPACE;
+
+  const size_t n = (size_t)B * H;
+  const Range rq = range_of(q, n * T * dk * e), rk = range_of(k, n * T * dk * e),
+              rv = range_of(v, n * T * dv * e), rg = range_of(g, n * T * dk * e),
+              rb = range_of(beta, n * T * e), rh0 = range_of(h0, h0 ? n * dk * dv * 4 : 0),
+              ro = range_of(o, n * T * dv * e), rhT = range_of(h_T, h_T ? n * dk * dv * 4 : 0),
+              rw = range_of(workspace, plan.workspace);
+  const Range ins[] = {rq, rk, rv, rg, rb, rh0};
+  for (const Range &r : ins)
+    if (overlap(ro, r)) return KDA_ERR_ALIAS;
+  for (int i = 0; i < 5; ++i)
+    if (overlap(rhT, ins[i])) return KDA_ERR_ALIAS;
+  if (h_T && h0 && overlap(rhT, rh0) && (const void *)h_T != (const void *)h0) return KDA_ERR_ALIAS;
+  if (overlap(rhT, ro)) return KDA_ERR_ALIAS;
+  for (const Range &r : ins)
+    if (overlap(rw, r)) return KDA_ERR_ALIAS;
+  if (overlap(rw, ro) || overlap(rw, rhT)) return KDA_ERR_ALIAS;
+
+  st = check_device();
+  if (st != KDA_OK) return st;
+
+  kda::ChunkArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0; a.o = o; a.hT = h_T;
+  a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv;
+  a.bf16 = dtype == KDA_DTYPE_BF16;
+  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
+  a.status = kda::device_status_ptr();
+  if (!a.status) return KDA_ERR_CUDA;
+  if (T == 0 && !h_T) return KDA_OK;
+  const cudaError_t ce = kda::launch_chunk_simt16(a, (cudaStream_t)stream);
+  return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, float *S, void *o, int B, int H, int dk, int dv,
+                                kda_dtype_t dtype, float scale, kda_stream_t stream) {
+  if (B < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (B * H == 0) return KDA_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+  const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(S)) return KDA_ERR_ALIGNMENT;
+  const void *ptrs[] = {q, k, v, g, beta, o};
+  for (const void *p : ptrs)
+    if (((uintptr_t)p % e) != 0) return KDA_ERR_ALIGNMENT;
+  const size_t n = (size_t)B * H;
+  const Range rq = range_of(q, n * dk * e), rk = range_of(k, n * dk * e), rv = range_of(v, n * dv * e),
+              rg = range_of(g, n * dk * e), rb = range_of(beta, n * e),
+              rS = range_of(S, n * dk * dv * 4), ro = range_of(o, n * dv * e);
+  const Range ins[] = {rq, rk, rv, rg, rb};
+  for (const Range &r : ins)
+    if (overlap(ro, r) || overlap(rS, r)) return KDA_ERR_ALIAS;
+  if (overlap(ro, rS)) return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  kda::DecodeArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
+  a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+  a.bf16 = dtype == KDA_DTYPE_BF16;
+  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
+  const cudaError_t ce = kda::launch_recurrent_step(a, (cudaStream_t)stream);
+  return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_get_device_status(kda_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+  unsigned *p = kda::device_status_ptr();
+  if (!p) return KDA_ERR_CUDA;
+  unsigned w = 0;
+  if (cudaMemcpy(&w, p, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+  if (w != kda::kDevOk) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  if (w == kda::kDevTimeout) return KDA_ERR_TIMEOUT;
+  if (w != kda::kDevOk) return KDA_ERR_DEVICE;
+  return KDA_OK;
+}
+
+}  // extern "C"

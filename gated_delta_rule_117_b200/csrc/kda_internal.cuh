@@ -1,0 +1,39 @@
+// Internal launch interface between the C-ABI layer (kda_api.cu) and the
+// kernels.  Not installed; the public interface is include/kda.h.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Device status word codes (written by kernels, read by kda_get_device_status).
+enum : unsigned { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
+
+// Address of the status word on the current device.
+unsigned *device_status_ptr();
+
+struct ChunkArgs {
+  const void *q, *k, *v, *g, *beta;
+  const float *h0;
+  void *o;
+  float *hT;
+  int B, H, T, dk, dv;
+  int bf16;     // 1: q,k,v,g,beta,o are bf16; 0: fp32
+  float scale;  // resolved (> 0)
+  unsigned *status;
+};
+
+struct DecodeArgs {
+  const void *q, *k, *v, *g, *beta;
+  float *S;
+  void *o;
+  int B, H, dk, dv;
+  int bf16;
+  float scale;
+};
+
+cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_recurrent_step(const DecodeArgs &a, cudaStream_t s);
+
+}  // namespace kda

@@ -1,0 +1,177 @@
+"""ctypes binding of libkda (include/kda.h).
+
+Argument marshalling only: the raw functions carry the C names and take
+integer device pointers; the torch helpers below turn tensors into those
+pointers and the current CUDA stream.  Every step of the computation runs in
+libkda's kernels.  There is no fallback: if ``libkda.so`` is missing or the
+device is unsupported, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+SO = os.path.join(PKG, "libkda.so")
+
+KDA_OK = 0
+KDA_DTYPE_F32 = 0
+KDA_DTYPE_BF16 = 1
+KDA_PATH_AUTO, KDA_PATH_SIMT16, KDA_PATH_TC64 = 0, 1, 2
+STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE", "KDA_ERR_ALIGNMENT",
+                "KDA_ERR_ALIAS", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT",
+                "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
+EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
+            "kda_status_string", "kda_get_device_status", "kda_version"]
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__("%s%s" % (kda_status_string(status), (" (" + what + ")") if what else ""))
+
+
+class kda_plan_t(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("chunk_size", ctypes.c_int), ("segments", ctypes.c_int),
+                ("launches", ctypes.c_int), ("workspace", ctypes.c_size_t)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library():
+    """Load libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(SO):
+                raise RuntimeError("libkda.so is not built (run gated_delta_rule_117_b200.build.build())")
+            lib = ctypes.CDLL(SO)
+            vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            lib.kda_chunk_fwd_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(kda_plan_t)]
+            lib.kda_chunk_fwd_plan.restype = i
+            lib.kda_chunk_fwd_workspace_size.argtypes = [i] * 7
+            lib.kda_chunk_fwd_workspace_size.restype = sz
+            lib.kda_chunk_fwd.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
+            lib.kda_chunk_fwd.restype = i
+            lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
+            lib.kda_recurrent_step.restype = i
+            lib.kda_status_string.argtypes = [i]
+            lib.kda_status_string.restype = ctypes.c_char_p
+            lib.kda_get_device_status.argtypes = [vp]
+            lib.kda_get_device_status.restype = i
+            lib.kda_version.argtypes = []
+            lib.kda_version.restype = i
+            _lib = lib
+    return _lib
+
+
+# ---- raw C-ABI calls (integer pointers) ------------------------------------
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return load_library().kda_version()
+
+
+def kda_chunk_fwd_plan(B, H, T, dk, dv, dtype, chunk_size=0):
+    p = kda_plan_t()
+    st = load_library().kda_chunk_fwd_plan(B, H, T, dk, dv, dtype, chunk_size, ctypes.byref(p))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_plan")
+    return dict(path=p.path, chunk_size=p.chunk_size, segments=p.segments, launches=p.launches,
+                workspace=p.workspace)
+
+
+def kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dtype, chunk_size=0) -> int:
+    return load_library().kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dtype, chunk_size)
+
+
+def kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale,
+                  workspace, workspace_bytes, stream) -> int:
+    """Returns the raw kda_status_t."""
+    return load_library().kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size,
+                                        scale, workspace, workspace_bytes, stream)
+
+
+def kda_recurrent_step(q, k, v, g, beta, S, o, B, H, dk, dv, dtype, scale, stream) -> int:
+    return load_library().kda_recurrent_step(q, k, v, g, beta, S, o, B, H, dk, dv, dtype, scale, stream)
+
+
+def kda_get_device_status(stream=None) -> int:
+    return load_library().kda_get_device_status(stream)
+
+
+# ---- torch helpers ---------------------------------------------------------
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError("q/k/v/g/beta must be bf16 or fp32, got %s" % t.dtype)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libkda takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libkda takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, h_T=None, scale=0.0, chunk_size=0,
+              output_final_state=True, workspace=None, stream=None):
+    """Prefill over [B, H, T, d] tensors (see kda_chunk_fwd in include/kda.h).
+
+    Allocates o / h_T / workspace with torch when not given.  Returns (o, h_T).
+    """
+    import torch
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_T is None and output_final_state:
+        h_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    ws = kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dt, chunk_size)
+    if ws == (1 << 64) - 1:
+        raise KdaError(2, "kda_chunk_fwd_workspace_size")
+    if ws > 0 and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    st = kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(h_T),
+                       B, H, T, dk, dv, dt, chunk_size, float(scale), _ptr(workspace),
+                       0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd")
+    return o, h_T
+
+
+def recurrent_step(q, k, v, g, beta, S, *, o=None, scale=0.0, stream=None):
+    """One decode step over [B, H, d] tensors; S [B, H, dk, dv] fp32 updated in place.  Returns o."""
+    import torch
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    st = kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), B, H, dk, dv,
+                            _dtype_code(q), float(scale), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_recurrent_step")
+    return o

@@ -1,0 +1,158 @@
+/*
+ * libkda -- Kimi Delta Attention (KDA) forward pass on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (Kimi K3 technical report, section 2.1.1, Eq. 1 and Eq. 5):
+ * per (batch b, head h) chain a state S_t in R^{dk x dv} evolves as
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = scale * S_t^T q_t,          alpha_t = exp(g_t)  (per key channel),
+ *
+ * where g_t in R^{dk} is the per-channel LOG-decay (the report's lower-bounded
+ * gate g = g_min * Sigmoid(e^A z), g_min = -5, keeps g in (-5, 0); the library
+ * takes g as an input and relies on g <= 0 and on every 16-token window sum of
+ * g staying >= -80, which that gate guarantees) and beta_t in (0, 1) is the
+ * delta-rule write strength.  The output reads the post-update state.  The
+ * report's Eq. 1 has no output scale; this library applies `scale` to o only
+ * (default dk^-1/2), never to the state.
+ *
+ * Prefill evaluates the chunkwise-parallel form of the report (section 2.1.1,
+ * Eqs. 3-4: cumulative decay, UT transform, intra/inter-chunk outputs, state
+ * carried across chunks); decode applies Eq. 1 to one token per sequence with
+ * the state updated in place (section 5.4.2).  Both are mathematically the
+ * same recurrence; results differ from an exact evaluation only by rounding.
+ *
+ * Conventions for every entry point
+ *  - All tensor arguments are DEVICE pointers to dense row-major (contiguous)
+ *    arrays owned by the caller.  libkda never allocates, frees or retains
+ *    them, and keeps no per-call state.  Alignment: every fp32 state pointer
+ *    (h0, h_T, S) and every prefill q, k, v, g, o and workspace pointer must be
+ *    16-byte aligned; beta and the decode q, k, v, g, o need only be aligned
+ *    to their element size.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without synchronising.  Argument errors are
+ *    detected synchronously, before anything is enqueued; a failed launch
+ *    returns KDA_ERR_CUDA.  Errors raised on the device (a bounded wait that
+ *    gave up) are recorded in a device status word read by
+ *    kda_get_device_status().
+ *  - Thread-safe: no global mutable host state besides a per-device cache of
+ *    the status-word address filled on first use.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef LIBKDA_KDA_H_
+#define LIBKDA_KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* NULL required pointer, bad scale, negative size */
+  KDA_ERR_SHAPE = 2,       /* unsupported B/H/T/dk/dv/chunk combination */
+  KDA_ERR_DTYPE = 3,       /* unknown kda_dtype_t, or dtype not supported by the requested path */
+  KDA_ERR_ALIGNMENT = 4,   /* a pointer breaks the alignment rule above */
+  KDA_ERR_ALIAS = 5,       /* an output overlaps an input (other than the allowed in-place cases) */
+  KDA_ERR_WORKSPACE = 6,   /* workspace missing or smaller than the size query returned */
+  KDA_ERR_CUDA = 7,        /* a CUDA runtime call or kernel launch failed */
+  KDA_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (see kda_get_device_status) */
+  KDA_ERR_UNSUPPORTED = 9, /* device is not sm_100 / path not available */
+  KDA_ERR_DEVICE = 10      /* device-side bounds check failed (see kda_get_device_status) */
+} kda_status_t;
+
+typedef enum {
+  KDA_DTYPE_F32 = 0, /* fp32 q, k, v, g, beta, o */
+  KDA_DTYPE_BF16 = 1 /* bf16 q, k, v, g, beta, o (state and accumulation stay fp32) */
+} kda_dtype_t;
+
+/* Kernel families selectable for prefill (see kda_chunk_fwd). */
+typedef enum {
+  KDA_PATH_AUTO = 0,   /* library choice */
+  KDA_PATH_SIMT16 = 1, /* fp32 CUDA-core chunked kernel, 16-token chunks, any supported dtype/d */
+  KDA_PATH_TC64 = 2    /* tcgen05 tensor-core chunked kernel, 64-token chunks, bf16, dk = dv = 128 */
+} kda_path_t;
+
+/* What kda_chunk_fwd will launch for a given problem (for benchmarks/tests). */
+typedef struct {
+  int path;         /* kda_path_t actually used */
+  int chunk_size;   /* tokens per chunk of the chosen kernel */
+  int segments;     /* in-device context-parallel segments per chain (1 = none) */
+  int launches;     /* kernel launches per call */
+  size_t workspace; /* bytes of workspace the call needs */
+} kda_plan_t;
+
+/*
+ * Plan a prefill call (no device work).  chunk_size selects the kernel:
+ * 0 = automatic, 16 = KDA_PATH_SIMT16, 64 = KDA_PATH_TC64.  Returns KDA_OK and
+ * fills *plan, or the error kda_chunk_fwd would return for these sizes.
+ */
+kda_status_t kda_chunk_fwd_plan(int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                int chunk_size, kda_plan_t *plan);
+
+/* Workspace bytes kda_chunk_fwd needs (0 if none, (size_t)-1 on invalid sizes). */
+size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                    int chunk_size);
+
+/*
+ * Prefill / training forward over T tokens for B x H independent chains
+ * (Kimi K3 report, section 2.1.1, Eqs. 1-4; in-device context parallelism of
+ * section 5.1.1 for long chains).
+ *
+ *   q, k, g : [B, H, T, dk]  dtype         g = per-channel log-decay (<= 0)
+ *   v       : [B, H, T, dv]  dtype
+ *   beta    : [B, H, T]      dtype
+ *   h0      : [B, H, dk, dv] fp32, or NULL for a zero initial state
+ *   o       : [B, H, T, dv]  dtype (written; bf16 outputs are rounded to nearest even)
+ *   h_T     : [B, H, dk, dv] fp32 final state, or NULL if not wanted.
+ *             h_T == h0 (exactly the same pointer) is allowed: in-place carry.
+ *   dk, dv  : each one of 16, 32, 64, 128 (KDA_PATH_TC64: both 128)
+ *   T       : >= 0 (T = 0 copies h0, or zeros, to h_T); need not be a
+ *             multiple of the chunk size
+ *   scale   : output scale; <= 0 selects dk^-1/2; must be finite
+ *   workspace, workspace_bytes : device scratch of at least
+ *             kda_chunk_fwd_workspace_size(...) bytes (may be NULL when that is 0);
+ *             contents on entry are ignored, on exit undefined
+ * o must not overlap any input, and
+ * h_T must not overlap any input except by being identical to h0.
+ */
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
+                           const void *beta, const float *h0, void *o, float *h_T, int B, int H,
+                           int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
+                           void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * One recurrent decode step, one new token per sequence (Kimi K3 report,
+ * Eq. 1 applied once; section 5.4.2: the state is updated in place).
+ *
+ *   q, k, g : [B, H, dk] dtype;  v : [B, H, dv] dtype;  beta : [B, H] dtype
+ *   S       : [B, H, dk, dv] fp32, read and overwritten in place with S_t
+ *   o       : [B, H, dv] dtype (written)
+ *   dk, dv  : each one of 16, 32, 64, 128;  scale as for kda_chunk_fwd.
+ * o must not overlap S or any input; S must not overlap any input.
+ */
+kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, float *S, void *o, int B, int H, int dk, int dv,
+                                kda_dtype_t dtype, float scale, kda_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status_t s);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's status word
+ * that kernels set when a bounded wait gives up (KDA_ERR_TIMEOUT) or a
+ * device-side check fails (KDA_ERR_DEVICE).  Returns KDA_OK if nothing was
+ * recorded, KDA_ERR_CUDA if synchronising failed.
+ */
+kda_status_t kda_get_device_status(kda_stream_t stream);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBKDA_KDA_H_ */

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function include/kda.h declares, plans calls, and rejects bad arguments
+synchronously with the documented status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gated_delta_rule_117_b200 import build as kbuild
+from gated_delta_rule_117_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "kda_chunk_fwd" in names and "kda_recurrent_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kda.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(kda.STATUS_NAMES):
+        assert kda.kda_status_string(code).startswith(name)
+    assert kda.kda_status_string(999) == "KDA_ERR_UNKNOWN"
+    assert kda.kda_version() >= 100
+
+
+def test_plan(lib):
+    p = kda.kda_chunk_fwd_plan(1, 2, 64, 16, 16, kda.KDA_DTYPE_F32, 16)
+    assert p["chunk_size"] == 16 and p["launches"] == 1 and p["segments"] >= 1
+    with pytest.raises(kda.KdaError) as e:
+        kda.kda_chunk_fwd_plan(1, 2, 64, 24, 16, kda.KDA_DTYPE_F32, 0)
+    assert e.value.status == 2
+    assert kda.kda_chunk_fwd_workspace_size(1, 2, 64, 24, 16, 0, 0) == (1 << 64) - 1
+
+
+# Fake, never-dereferenced device addresses: validation must reject bad
+# arguments before any CUDA call.
+BASE = 1 << 40
+N = 1 * 2 * 64 * 16 * 4  # bytes of one [1, 2, 64, 16] fp32 tensor
+
+
+def _call(**over):
+    B, H, T, dk, dv = 1, 2, 64, 16, 16
+    n = N
+    a = dict(q=BASE, k=BASE + n, v=BASE + 2 * n, g=BASE + 3 * n, beta=BASE + 4 * n, h0=BASE + 5 * n,
+             o=BASE + 6 * n, h_T=BASE + 7 * n, B=B, H=H, T=T, dk=dk, dv=dv, dtype=0, chunk_size=16,
+             scale=0.0, workspace=None, workspace_bytes=0, stream=None)
+    a.update(over)
+    return kda.kda_chunk_fwd(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(T=-1), 1), (dict(scale=float("nan")), 1),
+    (dict(dk=24), 2), (dict(dv=256), 2), (dict(chunk_size=32), 2),
+    (dict(dtype=7), 3),
+    (dict(k=BASE + N + 2), 4), (dict(h0=BASE + 5 * N + 8), 4), (dict(beta=BASE + 4 * N + 2), 4),
+    (dict(o=BASE + 100 * 16), 5),           # o overlaps q
+    (dict(h_T=BASE + 3 * N), 5),            # h_T == g
+    (dict(h_T=BASE + 5 * N + 16), 5),       # h_T partially overlaps h0
+])
+def test_chunk_fwd_rejects(lib, over, code):
+    assert _call(**over) == code
+
+
+def test_chunk_fwd_allows_inplace_state(lib):
+    st = _call(h_T=BASE + 5 * N)
+    # valid arguments: on a machine without a GPU the call fails only at the device check
+    if not torch.cuda.is_available():
+        assert st in (7, 9)
+
+
+def test_chunk_fwd_empty_batch_is_noop(lib):
+    assert _call(B=0) == 0 and _call(H=0, q=None) == 0
+
+
+def _dcall(**over):
+    B, H, dk, dv = 4, 2, 16, 16
+    n = 4096
+    a = dict(q=BASE, k=BASE + n, v=BASE + 2 * n, g=BASE + 3 * n, beta=BASE + 4 * n, S=BASE + 5 * n,
+             o=BASE + 5 * n + B * H * dk * dv * 4, B=B, H=H, dk=dk, dv=dv, dtype=1, scale=0.0, stream=None)
+    a.update(over)
+    return kda.kda_recurrent_step(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(S=None), 1), (dict(B=-1), 1), (dict(scale=float("inf")), 1),
+    (dict(dk=8), 2), (dict(dtype=5), 3),
+    (dict(S=BASE + 5 * 4096 + 4), 4), (dict(beta=BASE + 4 * 4096 + 1), 4),
+    (dict(o=BASE + 5 * 4096), 5),   # o inside S
+    (dict(S=BASE + 2 * 4096), 5),   # S overlaps v..beta
+])
+def test_recurrent_step_rejects(lib, over, code):
+    assert _dcall(**over) == code
+
+
+def test_no_cpu_fallback_without_gpu(lib):
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert _dcall() in (7, 9)

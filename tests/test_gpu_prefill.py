@@ -1,0 +1,141 @@
+"""GPU parity of kda_chunk_fwd against the fp64 oracle on the same seeded
+inputs: relative L2 error <= 1e-5 for fp32 inputs and <= 3e-3 (o and h_T) for
+bf16 inputs, at small sizes spanning several chunks plus ragged tails, at the
+full workload sizes (oracle on sampled heads), and on the edge cases."""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_117_b200 import kda, synth
+from parity_util import TOL, f64, oracle_prefill, rel_l2, to_dev
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, chunk_size=0, use_h0=True, scale=0.0, **kw):
+    d = to_dev(x)
+    return kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"] if use_h0 else None,
+                         chunk_size=chunk_size, scale=scale, **kw)
+
+
+def test_tiny_f32_workload():
+    w = synth.WORKLOADS["tiny_f32"]
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x, chunk_size=w.chunk, use_h0=False)
+    o_ref, h_ref = oracle_prefill(x, h0=False)
+    assert rel_l2(o, o_ref) <= TOL["f32"]
+    assert rel_l2(hT, h_ref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 32), (128, 16), (16, 128), (128, 128)])
+@pytest.mark.parametrize("T", [1, 15, 16, 47, 130])
+def test_shapes_and_ragged_tails(dtype, dk, dv, T):
+    w = synth.WORKLOADS["tiny_f32"].with_(dtype=dtype, B=2, H=3, T=T, dk=dk, dv=dv, h0_std=0.02, seed=77)
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL[dtype]
+    assert rel_l2(hT, h_ref) <= TOL[dtype]
+
+
+def test_prefill_workload_reduced_T():
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=700)
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_prefill_workload_full():
+    w = synth.WORKLOADS["prefill_h16_t4k"]
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_batched_workload_full_sampled_heads():
+    w = synth.WORKLOADS["batched_b8_h32_t8k"]
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x, use_h0=False)
+    fast = synth.fast_decay_heads(w).tolist()
+    heads = [(0, 0), (3, fast[0]), (7, fast[-1]), (5, 17)]
+    o_ref, h_ref = oracle_prefill(x, heads=heads, h0=False)
+    ob = torch.stack([o[b, h] for b, h in heads]).cpu()
+    hb = torch.stack([hT[b, h] for b, h in heads]).cpu()
+    assert rel_l2(ob, o_ref) <= TOL["bf16"] and rel_l2(hb, h_ref) <= TOL["bf16"]
+    assert torch.isfinite(o).all() and torch.isfinite(hT).all()
+
+
+def test_long_workload_reduced_T():
+    w = synth.WORKLOADS["long_h16_t1m"].with_(T=1 << 15, H=4)
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x, use_h0=False)
+    o_ref, h_ref = oracle_prefill(x, h0=False)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_zero_length_copies_state():
+    w = synth.WORKLOADS["tiny_f32"].with_(T=0, h0_std=0.02)
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x)
+    assert o.numel() == 0 and torch.equal(hT.cpu(), x["h0"])
+    o, hT = _run(x, use_h0=False)
+    assert torch.count_nonzero(hT) == 0
+
+
+def test_inplace_state_and_no_final_state():
+    w = synth.WORKLOADS["tiny_f32"].with_(T=40, h0_std=0.02, dtype="bf16", dk=32, dv=32)
+    x = synth.prefill_inputs(w)
+    d = to_dev(x)
+    o_ref, h_ref = oracle_prefill(x)
+    h = d["h0"].clone()
+    o, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h, h_T=h)
+    assert hT.data_ptr() == h.data_ptr()
+    assert rel_l2(h, h_ref) <= TOL["bf16"] and rel_l2(o, o_ref) <= TOL["bf16"]
+    o2, none = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], output_final_state=False)
+    assert none is None and torch.equal(o2, o)
+
+
+def test_explicit_scale():
+    w = synth.WORKLOADS["tiny_f32"].with_(T=33, h0_std=0.02)
+    x = synth.prefill_inputs(w)
+    o, _ = _run(x, scale=0.5)
+    o_ref, _ = oracle_prefill(x, scale=0.5)
+    assert rel_l2(o, o_ref) <= TOL["f32"]
+
+
+def test_state_split_resume_on_gpu():
+    # run(T) == run(T1) then run(T - T1) from h_T1, on the device path itself
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=256, H=2)
+    x = synth.prefill_inputs(w)
+    d = to_dev(x)
+    o, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"])
+    T1 = 100
+    sl = lambda t, a, b: t[:, :, a:b].contiguous()
+    o1, h1 = kda.chunk_fwd(*(sl(d[n], 0, T1) for n in ("q", "k", "v", "g", "beta")), d["h0"])
+    o2, h2 = kda.chunk_fwd(*(sl(d[n], T1, 256) for n in ("q", "k", "v", "g", "beta")), h1)
+    assert rel_l2(torch.cat([o1, o2], 2), o.float()) <= 3e-3
+    assert rel_l2(h2, hT) <= 1e-4
+
+
+def test_deterministic():
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=300, H=4)
+    x = synth.prefill_inputs(w)
+    o1, h1 = _run(x)
+    o2, h2 = _run(x)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def test_misaligned_pointer_is_rejected():
+    w = synth.WORKLOADS["tiny_f32"].with_(T=16)
+    d = to_dev(synth.prefill_inputs(w))
+    buf = torch.empty(d["q"].numel() + 4, device="cuda")
+    qm = buf[1:1 + d["q"].numel()].view_as(d["q"])
+    with pytest.raises(kda.KdaError) as e:
+        kda.chunk_fwd(qm, d["k"], d["v"], d["g"], d["beta"], None)
+    assert e.value.status == 4
+    assert kda.kda_get_device_status() == 0
