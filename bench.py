@@ -137,6 +137,7 @@ def main():
     ap.add_argument("--chunk-size", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -166,6 +167,9 @@ def main():
     stream = torch.cuda.current_stream()
     pk, pk_kind = peaks()
 
+    if args.decode_only:
+        print(json.dumps(measure_decode(args, synth, kda, torch, dev, pk, pk_kind)))
+        return
     assert not w.decode, "main line is a prefill workload"
     x = synth.prefill_inputs(w)
     d = {k: v.to(dev) for k, v in x.items()}
