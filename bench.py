@@ -223,7 +223,7 @@ def main():
     achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9
     flops = synth.flops_per_token_head(dk, dv, 64) * B * H * T
     tflops = flops / (kern_ms / 1e3) / 1e12
-    kernel_name = "chunk16_kernel" if plan["path"] == kda.KDA_PATH_SIMT16 else "kda_tc64"
+    kernel_name = "chunk16_kernel" if plan["path"] == kda.KDA_PATH_SIMT16 else "chunk_tc_kernel"
     src = (["gated_delta_rule_117_b200/csrc/kda_chunk_simt.cu"] if plan["path"] == kda.KDA_PATH_SIMT16
            else ["gated_delta_rule_117_b200/csrc/kda_chunk_tc.cu"])
     trec = traffic_record("%s:%s" % (kernel_name, w.name), src)

@@ -67,11 +67,13 @@ kda_status_t plan_prefill(int B, int H, int T, int dk, int dv, kda_dtype_t dtype
   if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
   if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
   if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
-  if (chunk_size != 0 && chunk_size != 16 && chunk_size != 64) return KDA_ERR_SHAPE;
-  if (chunk_size == 64) return KDA_ERR_UNSUPPORTED;  // tensor-core path not built in this version
+  if (chunk_size != 0 && chunk_size != 16 && chunk_size != 32) return KDA_ERR_SHAPE;
+  const bool tc_ok = dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128;
+  if (chunk_size == 32 && !tc_ok) return dtype == KDA_DTYPE_BF16 ? KDA_ERR_SHAPE : KDA_ERR_DTYPE;
   kda_plan_t p;
-  p.path = KDA_PATH_SIMT16;
-  p.chunk_size = 16;
+  const bool tc = chunk_size == 32 || (chunk_size == 0 && tc_ok);
+  p.path = tc ? KDA_PATH_TC32 : KDA_PATH_SIMT16;
+  p.chunk_size = tc ? 32 : 16;
   p.segments = 1;
   p.launches = (B * H == 0) ? 0 : 1;
   p.workspace = 0;
@@ -160,7 +162,8 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
   a.status = kda::device_status_ptr();
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
-  const cudaError_t ce = kda::launch_chunk_simt16(a, (cudaStream_t)stream);
+  const cudaError_t ce = plan.path == KDA_PATH_TC32 ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
+                                                    : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
   return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

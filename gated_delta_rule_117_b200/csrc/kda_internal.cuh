@@ -34,6 +34,7 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_recurrent_step(const DecodeArgs &a, cudaStream_t s);
 
 }  // namespace kda

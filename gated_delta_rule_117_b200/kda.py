@@ -18,7 +18,7 @@ SO = os.path.join(PKG, "libkda.so")
 KDA_OK = 0
 KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
-KDA_PATH_AUTO, KDA_PATH_SIMT16, KDA_PATH_TC64 = 0, 1, 2
+KDA_PATH_AUTO, KDA_PATH_SIMT16, KDA_PATH_TC32 = 0, 1, 2
 STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE", "KDA_ERR_ALIGNMENT",
                 "KDA_ERR_ALIAS", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT",
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]

@@ -73,7 +73,7 @@ typedef enum {
 typedef enum {
   KDA_PATH_AUTO = 0,   /* library choice */
   KDA_PATH_SIMT16 = 1, /* fp32 CUDA-core chunked kernel, 16-token chunks, any supported dtype/d */
-  KDA_PATH_TC64 = 2    /* tcgen05 tensor-core chunked kernel, 64-token chunks, bf16, dk = dv = 128 */
+  KDA_PATH_TC32 = 2    /* tcgen05 tensor-core chunked kernel, 32-token chunks, bf16, dk = dv = 128 */
 } kda_path_t;
 
 /* What kda_chunk_fwd will launch for a given problem (for benchmarks/tests). */
@@ -87,7 +87,8 @@ typedef struct {
 
 /*
  * Plan a prefill call (no device work).  chunk_size selects the kernel:
- * 0 = automatic, 16 = KDA_PATH_SIMT16, 64 = KDA_PATH_TC64.  Returns KDA_OK and
+ * 0 = automatic (KDA_PATH_TC32 for bf16 with dk = dv = 128, else
+ * KDA_PATH_SIMT16), 16 = KDA_PATH_SIMT16, 32 = KDA_PATH_TC32.  Returns KDA_OK and
  * fills *plan, or the error kda_chunk_fwd would return for these sizes.
  */
 kda_status_t kda_chunk_fwd_plan(int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
@@ -109,9 +110,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dty
  *   o       : [B, H, T, dv]  dtype (written; bf16 outputs are rounded to nearest even)
  *   h_T     : [B, H, dk, dv] fp32 final state, or NULL if not wanted.
  *             h_T == h0 (exactly the same pointer) is allowed: in-place carry.
- *   dk, dv  : each one of 16, 32, 64, 128 (KDA_PATH_TC64: both 128)
+ *   dk, dv  : each one of 16, 32, 64, 128 (KDA_PATH_TC32: both 128, bf16 only)
  *   T       : >= 0 (T = 0 copies h0, or zeros, to h_T); need not be a
  *             multiple of the chunk size
+ *   chunk_size : 0, 16 or 32, as for kda_chunk_fwd_plan (the result does not
+ *             depend on it beyond rounding)
  *   scale   : output scale; <= 0 selects dk^-1/2; must be finite
  *   workspace, workspace_bytes : device scratch of at least
  *             kda_chunk_fwd_workspace_size(...) bytes (may be NULL when that is 0);

@@ -44,6 +44,11 @@ def test_status_strings(lib):
 def test_plan(lib):
     p = kda.kda_chunk_fwd_plan(1, 2, 64, 16, 16, kda.KDA_DTYPE_F32, 16)
     assert p["chunk_size"] == 16 and p["launches"] == 1 and p["segments"] >= 1
+    assert p["path"] == kda.KDA_PATH_SIMT16
+    p = kda.kda_chunk_fwd_plan(1, 16, 4096, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    assert p["path"] == kda.KDA_PATH_TC32 and p["chunk_size"] == 32
+    p = kda.kda_chunk_fwd_plan(1, 16, 4096, 128, 128, kda.KDA_DTYPE_F32, 0)
+    assert p["path"] == kda.KDA_PATH_SIMT16
     with pytest.raises(kda.KdaError) as e:
         kda.kda_chunk_fwd_plan(1, 2, 64, 24, 16, kda.KDA_DTYPE_F32, 0)
     assert e.value.status == 2
@@ -68,8 +73,8 @@ def _call(**over):
 
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(o=None), 1), (dict(T=-1), 1), (dict(scale=float("nan")), 1),
-    (dict(dk=24), 2), (dict(dv=256), 2), (dict(chunk_size=32), 2),
-    (dict(dtype=7), 3),
+    (dict(dk=24), 2), (dict(dv=256), 2), (dict(chunk_size=64), 2), (dict(chunk_size=32, dtype=1), 2),
+    (dict(dtype=7), 3), (dict(chunk_size=32), 3),
     (dict(k=BASE + N + 2), 4), (dict(h0=BASE + 5 * N + 8), 4), (dict(beta=BASE + 4 * N + 2), 4),
     (dict(o=BASE + 100 * 16), 5),           # o overlaps q
     (dict(h_T=BASE + 3 * N), 5),            # h_T == g
