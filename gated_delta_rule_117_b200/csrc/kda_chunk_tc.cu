@@ -12,26 +12,36 @@
 // ones included, are dense tensor-core products (the report's Fig. 3b point).
 // With S~ = Diag(e^rho) S (the entering state decayed to the reference):
 //     A  = Tril_incl(Qs Kc^T),  L = StrictTril(Diag(beta) Ks Kc^T)
-//     T  = (I + L)^-1 Diag(beta)               (fp32 forward substitution)
+//     T  = (I + L)^-1 Diag(beta)               (fp32 blocked substitution)
 //     U  = T V,  W~ = T Ks,  V~ = U - W~ S~     (pseudo-values)
 //     O  = scale (Qs S~ + A V~)
 //     S' = Diag(e^{G_31}) S + Diag(e^{G_31 - rho}) Kc^T V~
 // Every tensor-core product is issued "transposed" so that M = 128 is a
-// channel dimension (value channel e or key channel c) and the TMEM lane is
-// the channel an epilogue thread owns:
+// channel dimension and the TMEM lane is the channel an epilogue thread owns:
 //     Gram  D[r|32+r][j] = [Qs; Ks] Kc^T          (M = 128: rows 64..127 unused)
-//     U^T   D[e][r]      = V^T T^T
-//     W~^T  D[c][r]      = Ks^T T^T
+//     U^T   D[e][r]      = V^T T^T,   W~^T D[c][r] = Ks^T T^T
 //     V~^T  D[e][r]     -= S~^T W~^T               (negated A, accumulated onto U^T)
 //     O^T   D[e][r]      = S~^T Qs^T + V~^T A^T
 //     dS^T  D[e][c]      = V~^T Kc
-// (Qs, Ks, Kc, A and V~ enter the Gram, output and state-update products as
-// hi + lo bf16 pairs; see the shared-memory layout below.)
-// Thread e of the 128-thread CTA keeps column e of the fp32 master state S in
-// registers for the whole chain; S~^T is rebuilt in shared memory (bf16) each
-// chunk.  One CTA owns one (b, h) chain; the next chunk's q, k, v, g tiles are
-// fetched by TMA while the current chunk is processed.  Every wait is bounded
-// and reports KDA_ERR_TIMEOUT through the device status word.
+// Qs and Kc (Gram), A and V~ (output), V~ and Kc (state update) enter as
+// hi + lo bf16 pairs multiplied as hi*hi + lo*hi + hi*lo; without that their
+// bf16 rounding would dominate the error.
+//
+// Work split (the report's token-parallel stage vs head-parallel recurrence,
+// section 5.1.1, mapped onto one CTA per (b, h) chain), 8 warps:
+//   warps 0-3  chain:  thread e keeps column e of the fp32 state S in
+//                      registers; per chunk it writes S~^T, issues the V~/O
+//                      MMAs, turns V~^T into bf16 hi/lo operands, issues the
+//                      dS/O MMAs, applies the state update and stores the
+//                      output tile;
+//   warps 4-7  token:  one chunk ahead of the chain: TMA loads, cumulative
+//                      decay and rescaled operands, the Gram MMAs, A, L, the
+//                      triangular solve, the U/W~ MMAs and W~.
+// One elected thread per warpgroup issues its MMAs and TMA copies right after
+// the group's named barrier.  The two groups hand chunks over through
+// mbarriers; buffers the chain reads are double buffered by chunk parity.
+// Every wait is bounded; a wait that gives up sets the device status word and
+// the whole CTA drains without further MMAs.
 #include <cuda_bf16.h>
 
 #include "kda_internal.cuh"
@@ -45,37 +55,54 @@ using namespace sm100;
 
 constexpr int C = 32;     // tokens per chunk
 constexpr int D = 128;    // dk = dv
-constexpr int NT = 128;   // threads per CTA
+constexpr int NT = 256;   // 8 warps
 constexpr uint32_t kWaitLimit = 1u << 22;  // polls; seconds, far beyond any real wait
+constexpr uint32_t kBarChain = 1, kBarTok = 2;
 
-// Shared-memory layout (byte offsets from a 1024-aligned base).  A [rows x 64]
-// bf16 tile of 128-byte swizzled rows is a "half" (channel block 0 or 1).
-// Operands whose bf16 rounding would dominate the error (the Gram operands,
-// and V~ / Kc in the state update) are kept as hi + lo bf16 pairs and
-// multiplied as hi*hi + lo*hi + hi*lo.
-constexpr int kQK = 0;          // 2 x 16 KB: [Qs h0 | Ks h0 | Qs h1 | Ks h1] (hi), 4 KB each
-constexpr int kQKL = 32768;     // 16 KB: the lo parts, same layout
-constexpr int kKC = 49152;      // 8 KB: Kc hi [Kc h0 | Kc h1]
-constexpr int kKCL = 57344;     // 8 KB: Kc lo (also the readable tail of the QKL operand view)
-constexpr int kV = 65536;       // 2 x 8 KB: [V h0 | V h1]
-constexpr int kG = 81920;       // 2 x 8 KB: [g h0 | g h1]
-constexpr int kST = 98304;      // 32 KB: S~^T [e][c], half c-block 0 (16 KB) | half 1
-constexpr int kVT = 131072;     // 16 KB: V~^T hi [e][j] (K = 32: first 64 B of each row)
-constexpr int kVTL = 147456;    // 16 KB: V~^T lo
-constexpr int kWT = 163840;     // 8 KB: W~ [r][c], half 0 | half 1
-constexpr int kTH = 172032;     // 4 KB: T [r][s]
-constexpr int kAH = 176128;     // 4 KB: A hi [r][j]
-constexpr int kAL = 180224;     // 4 KB: A lo
-constexpr int kLf = 184320;     // fp32 L [32][33]
-constexpr int kVec = 188544;    // fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128]
-constexpr int kBeta = 190080;   // fp32 beta[32]
-constexpr int kBar = 190208;    // mbarriers: tma[2], mma
-constexpr int kTslot = 190272;  // TMEM base address
-constexpr int kSmemBytes = 190288 + 1024;
+// ---- shared memory (byte offsets from a 1024-aligned base) -------------------
+// "h0/h1" = channel blocks 0..63 / 64..127 of a [tokens x 128] bf16 tile stored
+// as 128-byte swizzled rows (TMA SWIZZLE_128B layout), 4 KB per 32 tokens.
+constexpr int kRawQK = 0;        // q h0 | q h1 | k h0 | k h1 (TMA)
+constexpr int kRawG = 16384;     // g h0 | g h1 (TMA)
+constexpr int kRawV = 24576;     // v h0 | v h1 (TMA; the U MMA reads it in place)
+constexpr int kQKH = 32768;      // [2]: Qs hi h0 | Ks hi h0 | Qs hi h1 | Ks hi h1
+constexpr int kQKL = 65536;      // Qs lo / Ks lo, same layout (Gram only)
+constexpr int kKCH = 81920;      // [2]: Kc hi h0 | h1
+constexpr int kKCL = 98304;      // [2]: Kc lo h0 | h1
+constexpr int kST = 114688;      // S~^T [e][c], K-halves of 16 KB (SW128)
+constexpr int kVTH = 147456;     // V~^T hi [e][j] (SW64, 64-byte rows)
+constexpr int kVTL = 155648;     // V~^T lo
+constexpr int kWT = 163840;      // [2]: W~ stored [c][r] (SW64), 8 KB each
+constexpr int kAH = 180224;      // [2]: A hi [r][j] (SW64), 2 KB each; A lo at +4096
+constexpr int kTT = 188416;      // T [r][s] (SW64)
+constexpr int kLf = 190464;      // fp32 L [32][33]
+constexpr int kNf = 194688;      // fp32 N = (I + L)^-1 [32][33]
+constexpr int kXf = 198912;      // fp32 scratch [16][17]
+constexpr int kFac = 200000;     // [2]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
+constexpr int kXch = 203072;     // fp32 rho[128], G_31 - rho[128]
+constexpr int kBeta = 204096;    // fp32 beta[32]
+constexpr int kBar = 204224;     // mbarriers
+constexpr int kMisc = 204480;    // TMEM base address, abort flag
+constexpr int kSmemBytes = 204496 + 1024;
+
+// barrier slots
+enum {
+  B_QKG = 0,   // q,k,g of the chunk landed (TMA)
+  B_V,         // v of the chunk landed (TMA)
+  B_GRAM,      // Gram MMAs done
+  B_UW,        // U, W~ MMAs done
+  B_WT0,       // [2] token: chunk ready for the chain (W~, U, operands, factors)
+  B_WT1,
+  B_V1,        // V~ and O-inter MMAs done
+  B_DS,        // dS and O-intra MMAs done
+  B_CD0,       // [2] chain finished with the chunk's buffers
+  B_CD1,
+  B_COUNT
+};
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t tG = 0, tU = 32, tW = 64, tO = 96, tDS = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t tG = 0, tU0 = 32, tW = 96, tO = 128, tDS = 256;
 
 struct TcParams {
   const __nv_bfloat16 *beta;
@@ -87,11 +114,173 @@ struct TcParams {
   float scale;
 };
 
-__device__ __forceinline__ float bf(const unsigned char *p) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+struct Ctx {
+  unsigned char *sm;
+  uint64_t *bar;
+  volatile int *abort;
+  unsigned *status;
+};
+
+// Bounded wait that also returns (false) as soon as another role aborted.
+__device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity) {
+  uint64_t *b = &x.bar[slot];
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(b, parity)) return true;
+    if (*x.abort) return false;
+  }
+  *x.abort = 1;
+  atomicExch(x.status, kDevTimeout);
+  return false;
 }
-__device__ __forceinline__ void stbf(unsigned char *p, float x) {
-  *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
+
+// hi/lo pair of (a, b): returns packed hi, writes packed lo.
+__device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
+  const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
+  lo = pack_bf16x2(a - __bfloat162float(ha), b - __bfloat162float(hb));
+  __nv_bfloat162 h;
+  h.x = ha;
+  h.y = hb;
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// ---- token stage: one chunk, 128 threads (tt = 0..127) ------------------------
+__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int t0, int T, const __nv_bfloat16 *beta) {
+  unsigned char *sm = x.sm;
+  const int pp = tt & 63, hf = tt >> 6;  // channel pair (2pp, 2pp+1), token half
+  const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
+  float xs0[16], xs1[16];
+  float G0 = 0.f, G1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int s = 16 * hf + i;
+    const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawG + h * 4096 + sw128_off(s, cc));
+    G0 += __bfloat162float(g2.x);
+    G1 += __bfloat162float(g2.y);
+    xs0[i] = G0;
+    xs1[i] = G1;
+  }
+  float *xch = reinterpret_cast<float *>(sm + kXch);
+  if (hf == 0) {
+    // tokens 0..15: x = G_s - G_15 (>= 0); G_15 = rho
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      xs0[i] -= G0;
+      xs1[i] -= G1;
+    }
+    xch[c0] = G0;
+    xch[c0 + 1] = G1;
+  } else {
+    // tokens 16..31: x = sum_{16..s} g (<= 0); the half's total is G_31 - rho
+    xch[128 + c0] = G0;
+    xch[128 + c0 + 1] = G1;
+  }
+  unsigned char *qkh = sm + kQKH + p * 16384;
+  unsigned char *kch = sm + kKCH + p * 8192, *kcl = sm + kKCL + p * 8192;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int s = 16 * hf + i;
+    const float x0 = fminf(fmaxf(xs0[i], -87.f), 87.f), x1 = fminf(fmaxf(xs1[i], -87.f), 87.f);
+    const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
+    const uint32_t off = sw128_off(s, cc);
+    const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawQK + h * 4096 + off);
+    const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawQK + 8192 + h * 4096 + off);
+    const float q0 = __bfloat162float(q2.x), q1 = __bfloat162float(q2.y);
+    const float k0 = __bfloat162float(k2.x), k1 = __bfloat162float(k2.y);
+    uint32_t lo;
+    *reinterpret_cast<uint32_t *>(qkh + h * 8192 + off) = split2(q0 * e0, q1 * e1, lo);
+    *reinterpret_cast<uint32_t *>(sm + kQKL + h * 8192 + off) = lo;
+    *reinterpret_cast<uint32_t *>(qkh + h * 8192 + 4096 + off) = split2(k0 * e0, k1 * e1, lo);
+    *reinterpret_cast<uint32_t *>(sm + kQKL + h * 8192 + 4096 + off) = lo;
+    *reinterpret_cast<uint32_t *>(kch + h * 4096 + off) = split2(k0 * i0, k1 * i1, lo);
+    *reinterpret_cast<uint32_t *>(kcl + h * 4096 + off) = lo;
+  }
+  if (tt < C) {
+    float *bet = reinterpret_cast<float *>(sm + kBeta);
+    bet[tt] = (t0 + tt < T) ? __bfloat162float(beta[t0 + tt]) : 0.f;
+  }
+  named_sync(kBarTok, 128);
+  {
+    const int c = tt;
+    float *fac = reinterpret_cast<float *>(sm + kFac + p * 1536);
+    const float rho = xch[c], tail = xch[128 + c];
+    fac[c] = __expf(rho);                // e^rho
+    fac[128 + c] = __expf(rho + tail);   // e^{G_31}
+    fac[256 + c] = __expf(tail);         // e^{G_31 - rho}
+  }
+}
+
+// N = (I + L)^-1 for the strictly lower 32x32 L in Lf (fp32), blocked 8 -> 16 -> 32,
+// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  128 threads.
+__device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
+  unsigned char *sm = x.sm;
+  const float *L = reinterpret_cast<const float *>(sm + kLf);
+  float *N = reinterpret_cast<float *>(sm + kNf);
+  float *X = reinterpret_cast<float *>(sm + kXf);
+  const float *bet = reinterpret_cast<const float *>(sm + kBeta);
+  // level 1: the four 8x8 diagonal blocks, one column per thread
+  if (tt < 32) {
+    const int q = tt >> 3, jj = tt & 7, b0 = 8 * q;
+    float n[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      float acc = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+      for (int s = 0; s < r; ++s) acc -= L[(b0 + r) * 33 + b0 + s] * n[s];
+      n[r] = acc;
+      N[(b0 + r) * 33 + b0 + jj] = acc;
+    }
+  }
+  named_sync(kBarTok, 128);
+  // level 2: N_10 = -N_11 L_10 N_00 inside each 16x16 block (8x8 pieces)
+  {
+    const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) acc += L[(o + 8 + r) * 33 + o + s] * N[(o + s) * 33 + o + j];
+    X[blk * 64 + e] = acc;
+  }
+  named_sync(kBarTok, 128);
+  {
+    const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) acc += N[(o + 8 + r) * 33 + o + 8 + s] * X[blk * 64 + s * 8 + j];
+    N[(o + 8 + r) * 33 + o + j] = -acc;
+  }
+  named_sync(kBarTok, 128);
+  // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (2 elements per thread)
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) acc += L[(16 + r) * 33 + s] * N[s * 33 + j];
+    X[r * 17 + j] = acc;
+  }
+  named_sync(kBarTok, 128);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) acc += N[(16 + r) * 33 + 16 + s] * X[s * 17 + j];
+    N[(16 + r) * 33 + j] = -acc;
+  }
+  named_sync(kBarTok, 128);
+  // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 8-column chunk k)
+  {
+    const int r = tt >> 2, k = tt & 3;
+    uint4 w;
+    uint32_t *pw = &w.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j0 = 8 * k + 2 * i;
+      const float a0 = (j0 <= r) ? N[r * 33 + j0] * bet[j0] : 0.f;
+      const float a1 = (j0 + 1 <= r) ? N[r * 33 + j0 + 1] * bet[j0 + 1] : 0.f;
+      pw[i] = pack_bf16x2(a0, a1);
+    }
+    *reinterpret_cast<uint4 *>(sm + kTT + sw64_chunk(r, k)) = w;
+  }
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -100,14 +289,12 @@ __global__ void __launch_bounds__(NT, 1)
                     const TcParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + kBar);
-  uint64_t *bar_mma = bar_tma + 2;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kTslot);
-  float *Lf = reinterpret_cast<float *>(sm + kLf);
-  float *eRho = reinterpret_cast<float *>(sm + kVec);
-  float *eG31 = eRho + D;
-  float *decC = eG31 + D;
-  float *bet = reinterpret_cast<float *>(sm + kBeta);
+  Ctx x;
+  x.sm = sm;
+  x.bar = reinterpret_cast<uint64_t *>(sm + kBar);
+  x.abort = reinterpret_cast<volatile int *>(sm + kMisc + 4);
+  x.status = p.status;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x;
@@ -116,320 +303,293 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sbase = smem_u32(sm);
 
   if (tid == 0) {
-    mbar_init(&bar_tma[0], 1);
-    mbar_init(&bar_tma[1], 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&x.bar[i], 1);
+    *x.abort = 0;
     mbar_init_fence();
-    prefetch_tmap(&mq);
-    prefetch_tmap(&mk);
-    prefetch_tmap(&mv);
-    prefetch_tmap(&mg);
   }
-  if (warp == 0) {
+  if (warp == 4) {
     tmem_alloc(tslot, kTmemCols);
     tmem_relinquish();
-  }
-  // Master state: thread e holds S[c][e] for every key channel c.
-  float S[D];
-  {
-    const float *h0 = p.h0 ? p.h0 + (size_t)bh * D * D : nullptr;
-#pragma unroll
-    for (int c = 0; c < D; ++c) S[c] = h0 ? h0[c * D + tid] : 0.f;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const uint32_t tlane = tbase + ((uint32_t)(32 * warp) << 16);
 
-  auto issue_tma = [&](int t, int buf) {
-    unsigned char *qk = sm + kQK + buf * 16384;
-    unsigned char *vv = sm + kV + buf * 8192;
-    unsigned char *gg = sm + kG + buf * 8192;
-    mbar_arrive_expect_tx(&bar_tma[buf], 8 * 4096);
-    const int y = t * C;
-    tma_load_3d(qk, &mq, &bar_tma[buf], 0, y, bh);
-    tma_load_3d(qk + 8192, &mq, &bar_tma[buf], 64, y, bh);
-    tma_load_3d(qk + 4096, &mk, &bar_tma[buf], 0, y, bh);
-    tma_load_3d(qk + 12288, &mk, &bar_tma[buf], 64, y, bh);
-    tma_load_3d(vv, &mv, &bar_tma[buf], 0, y, bh);
-    tma_load_3d(vv + 4096, &mv, &bar_tma[buf], 64, y, bh);
-    tma_load_3d(gg, &mg, &bar_tma[buf], 0, y, bh);
-    tma_load_3d(gg + 4096, &mg, &bar_tma[buf], 64, y, bh);
-  };
-
-  // Chunks whose TMA was issued / whose TMA barrier was waited (thread 0's
-  // view is the one that matters for the abort path).
-  int tma_issued = 0, tma_waited = 0;
-  if (tid == 0 && nchunks > 0) issue_tma(0, 0);
-  tma_issued = nchunks > 0 ? 1 : 0;
-  uint32_t mma_phase = 0;
-  bool abort = false;
-
-  auto wait_mma = [&]() -> bool {
-    const bool ok = mbar_wait(bar_mma, mma_phase, kWaitLimit);
-    mma_phase ^= 1u;
-    tc_fence_after();
-    return __syncthreads_and(ok);
-  };
-  auto release_to_mma = [&]() {  // smem writes -> async proxy, TMEM reads done -> MMA may reuse
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  };
-
-  for (int t = 0; t < nchunks && !abort; ++t) {
-    const int b = t & 1;
-    const int t0 = t * C;
-    unsigned char *qk = sm + kQK + b * 16384;
-    unsigned char *gg = sm + kG + b * 8192;
-    if (t + 1 < nchunks) {
-      if (tid == 0) issue_tma(t + 1, b ^ 1);
-      tma_issued = t + 2;
-    }
+  if (warp < 4) {
+    // ======================= chain warpgroup =======================
+    const int e = tid;
+    const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
+    const uint32_t idV = idesc_bf16(128, 32, false, true, true);   // -S~^T W~^T (B MN-major)
+    const uint32_t idO = idesc_bf16(128, 32, false, false, false);
+    const uint32_t idS = idesc_bf16(128, 128, false, true, false);
+    float S[D];
     {
-      const bool ok = mbar_wait(&bar_tma[b], (uint32_t)(t >> 1) & 1u, kWaitLimit);
-      if (!__syncthreads_and(ok)) { abort = true; break; }
-      tma_waited = t + 1;
-    }
-
-    // ---- a-1: chunk-local cumulative log-decay and the rescaled operands -----
-    {
-      const int c = tid, h = c >> 6, cc = c & 63;
-      float Gs[C];
-      float G = 0.f;
+      const float *h0 = p.h0 ? p.h0 + (size_t)bh * D * D : nullptr;
 #pragma unroll
-      for (int s = 0; s < C; ++s) {
-        G += bf(gg + h * 4096 + sw128_off(s, cc));
-        Gs[s] = G;
-      }
-      const float rho = Gs[15], G31 = Gs[C - 1];
-#pragma unroll
-      for (int s = 0; s < C; ++s) {
-        const float x = fminf(fmaxf(Gs[s] - rho, -87.f), 87.f);
-        const float ex = expf(x), ix = expf(-x);
-        unsigned char *pq = qk + h * 8192 + sw128_off(s, cc);
-        unsigned char *pk = pq + 4096;
-        const float qv = bf(pq), kv = bf(pk);
-        const float qs = qv * ex, ksv = kv * ex, kc = kv * ix;
-        const __nv_bfloat16 qh = __float2bfloat16_rn(qs), kh = __float2bfloat16_rn(ksv), ch = __float2bfloat16_rn(kc);
-        const uint32_t off = h * 4096 + sw128_off(s, cc);
-        *reinterpret_cast<__nv_bfloat16 *>(pq) = qh;
-        *reinterpret_cast<__nv_bfloat16 *>(pk) = kh;
-        *reinterpret_cast<__nv_bfloat16 *>(sm + kKC + off) = ch;
-        stbf(sm + kQKL + h * 8192 + sw128_off(s, cc), qs - __bfloat162float(qh));
-        stbf(sm + kQKL + h * 8192 + 4096 + sw128_off(s, cc), ksv - __bfloat162float(kh));
-        stbf(sm + kKCL + off, kc - __bfloat162float(ch));
-      }
-      eRho[c] = expf(rho);
-      eG31[c] = expf(G31);
-      decC[c] = expf(G31 - rho);
-      if (tid < C) bet[tid] = (t0 + tid < T) ? __bfloat162float(p.beta[(size_t)bh * T + t0 + tid]) : 0.f;
+      for (int c = 0; c < D; ++c) S[c] = h0 ? h0[c * D + e] : 0.f;
     }
-    __syncthreads();
-    // ---- S~^T = (Diag(e^rho) S)^T in bf16: thread e writes row e -------------
-    {
-      const int e = tid;
+    for (int t = 0; t < nchunks; ++t) {
+      const int pb = t & 1, t0 = t * C;
+      const bool ready = wait_bar(x, B_WT0 + pb, (uint32_t)(t >> 1) & 1u);
+      const float *fac = reinterpret_cast<const float *>(sm + kFac + pb * 1536);
+      // S~^T(t): row e, c-blocks 0/1, eight 16-byte chunks each
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          uint4 w;
           const int c0 = h * 64 + k * 8;
-          w.x = pack_bf16x2(eRho[c0 + 0] * S[c0 + 0], eRho[c0 + 1] * S[c0 + 1]);
-          w.y = pack_bf16x2(eRho[c0 + 2] * S[c0 + 2], eRho[c0 + 3] * S[c0 + 3]);
-          w.z = pack_bf16x2(eRho[c0 + 4] * S[c0 + 4], eRho[c0 + 5] * S[c0 + 5]);
-          w.w = pack_bf16x2(eRho[c0 + 6] * S[c0 + 6], eRho[c0 + 7] * S[c0 + 7]);
+          uint4 w;
+          w.x = pack_bf16x2(fac[c0 + 0] * S[c0 + 0], fac[c0 + 1] * S[c0 + 1]);
+          w.y = pack_bf16x2(fac[c0 + 2] * S[c0 + 2], fac[c0 + 3] * S[c0 + 3]);
+          w.z = pack_bf16x2(fac[c0 + 4] * S[c0 + 4], fac[c0 + 5] * S[c0 + 5]);
+          w.w = pack_bf16x2(fac[c0 + 6] * S[c0 + 6], fac[c0 + 7] * S[c0 + 7]);
           *reinterpret_cast<uint4 *>(sm + kST + h * 16384 + sw128_chunk(e, k)) = w;
         }
-    }
-    release_to_mma();
-    // ---- a-2 Gram [Qs; Ks] Kc^T and the inter-chunk output S~^T Qs^T --------
-    if (tid == 0) {
-      const uint32_t qkA = sbase + kQK + b * 16384;
-      const uint32_t idG = idesc_bf16(128, 32, false, false, false);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_sync(kBarChain, 128);
+      if (e == 0 && ready && !*x.abort) {
+        tc_fence_after();
+        const uint32_t st = sbase + kST, wt = sbase + kWT + pb * 8192, qkh = sbase + kQKH + pb * 16384;
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {  // hi*hi, lo*hi, hi*lo
-        const uint32_t aBase = part == 1 ? sbase + kQKL : qkA;
-        const uint32_t bBase = sbase + (part == 2 ? kKCL : kKC);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_bf16(tbase + tG, sdesc_sw128(aBase + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                   sdesc_sw128(bBase + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024), idG, part > 0 || ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_bf16(tbase + tO, sdesc_sw128(sbase + kST + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                 sdesc_sw128(qkA + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), idG, ks > 0);
-      mma_commit(bar_mma);
-    }
-    if (!wait_mma()) { abort = true; break; }
-    // ---- a-2/a-3: masks, A (hi/lo), L, then T = (I + L)^-1 Diag(beta) --------
-    if (warp == 0) {
-      float a[32];
-      tmem_ld32(tlane + tG, a);
-      tmem_ld_wait();
-      const int r = lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint4 hi, lo;
-        uint32_t *ph = &hi.x, *pl = &lo.x;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j0 = k * 8 + 2 * i;
-          const float a0 = (j0 <= r) ? a[j0] : 0.f, a1 = (j0 + 1 <= r) ? a[j0 + 1] : 0.f;
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-          ph[i] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-          pl[i] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t ad = sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          mma_bf16(tbase + tU0 + 32 * pb, ad, sdesc_sw64(wt + ks * 1024, 8192, 512), idV, true);
+          mma_bf16(tbase + tO, ad, sdesc_sw128(qkh + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), idO, ks > 0);
         }
-        *reinterpret_cast<uint4 *>(sm + kAH + sw128_chunk(r, k)) = hi;
-        *reinterpret_cast<uint4 *>(sm + kAL + sw128_chunk(r, k)) = lo;
+        mma_commit(&x.bar[B_V1]);
       }
-    } else if (warp == 1) {
-      float l[32];
-      tmem_ld32(tlane + tG, l);
-      tmem_ld_wait();
-      const int r = lane;
-      const float br = bet[r];
+      // V~^T(t) -> bf16 hi/lo operands
+      wait_bar(x, B_V1, (uint32_t)t & 1u);
+      tc_fence_after();
+      {
+        float v[32];
+        tmem_ld32(tl + tU0 + 32 * pb, v);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) Lf[r * 33 + j] = (j < r) ? br * l[j] : 0.f;
-    }
-    __syncthreads();
-    if (warp == 1) {
-      const int j = lane;
-      float n[C];
-#pragma unroll
-      for (int r = 0; r < C; ++r) {
-        float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int s = 0; s + 1 < r; s += 2) {
-          acc0 -= Lf[r * 33 + s] * n[s];
-          acc1 -= Lf[r * 33 + s + 1] * n[s + 1];
-        }
-        if (r & 1) acc0 -= Lf[r * 33 + r - 1] * n[r - 1];
-        n[r] = acc0 + acc1;
-      }
-      const float bj = bet[j];
-#pragma unroll
-      for (int r = 0; r < C; ++r) stbf(sm + kTH + sw128_off(r, j), n[r] * bj);
-    }
-    release_to_mma();
-    // ---- a-3: U^T = V^T T^T, W~^T = Ks^T T^T ---------------------------------
-    if (tid == 0) {
-      const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
-      const uint32_t vA = sbase + kV + b * 8192, ksA = sbase + kQK + b * 16384 + 4096;
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const uint64_t bd = sdesc_sw128(sbase + kTH + ks * 32, 16, 1024);
-        mma_bf16(tbase + tU, sdesc_sw128(vA + ks * 2048, 4096, 1024), bd, idMK, ks > 0);
-        mma_bf16(tbase + tW, sdesc_sw128(ksA + ks * 2048, 8192, 1024), bd, idMK, ks > 0);
-      }
-      mma_commit(bar_mma);
-    }
-    if (!wait_mma()) { abort = true; break; }
-    // ---- W~ to shared memory (K-major [r][c]) ---------------------------------
-    {
-      float w[32];
-      tmem_ld32(tlane + tW, w);
-      tmem_ld_wait();
-      const int c = tid, h = c >> 6, cc = c & 63;
-#pragma unroll
-      for (int r = 0; r < C; ++r) stbf(sm + kWT + h * 4096 + sw128_off(r, cc), w[r]);
-    }
-    release_to_mma();
-    // ---- a-4: V~^T = U^T - S~^T W~^T ------------------------------------------
-    if (tid == 0) {
-      const uint32_t idN = idesc_bf16(128, 32, false, false, true);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_bf16(tbase + tU, sdesc_sw128(sbase + kST + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                 sdesc_sw128(sbase + kWT + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024), idN, true);
-      mma_commit(bar_mma);
-    }
-    if (!wait_mma()) { abort = true; break; }
-    {
-      float v[32];
-      tmem_ld32(tlane + tU, v);
-      tmem_ld_wait();
-      const int e = tid;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint4 hi, lo;
-        uint32_t *ph = &hi.x, *pl = &lo.x;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float v0 = v[8 * k + 2 * i], v1 = v[8 * k + 2 * i + 1];
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-          ph[i] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-          pl[i] = pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
-        }
-        *reinterpret_cast<uint4 *>(sm + kVT + sw128_chunk(e, k)) = hi;
-        *reinterpret_cast<uint4 *>(sm + kVTL + sw128_chunk(e, k)) = lo;
-      }
-    }
-    release_to_mma();
-    // ---- a-4: dS^T = V~^T Kc, O^T += V~^T A^T ----------------------------------
-    if (tid == 0) {
-      const uint32_t idS = idesc_bf16(128, 128, false, true, false);
-      const uint32_t idO = idesc_bf16(128, 32, false, false, false);
-#pragma unroll
-      for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
-        const uint32_t aBase = sbase + (part == 1 ? kVTL : kVT);
-        const uint32_t kcB = sbase + (part == 2 ? kKCL : kKC);
-        const uint32_t aB = sbase + (part == 2 ? kAL : kAH);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const uint64_t ad = sdesc_sw128(aBase + ks * 32, 16, 1024);
-          mma_bf16(tbase + tDS, ad, sdesc_sw128(kcB + ks * 2048, 4096, 1024), idS, part > 0 || ks > 0);
-          mma_bf16(tbase + tO, ad, sdesc_sw128(aB + ks * 32, 16, 1024), idO, true);
+        for (int k = 0; k < 4; ++k) {
+          uint4 hi, lo;
+          hi.x = split2(v[8 * k + 0], v[8 * k + 1], lo.x);
+          hi.y = split2(v[8 * k + 2], v[8 * k + 3], lo.y);
+          hi.z = split2(v[8 * k + 4], v[8 * k + 5], lo.z);
+          hi.w = split2(v[8 * k + 6], v[8 * k + 7], lo.w);
+          *reinterpret_cast<uint4 *>(sm + kVTH + sw64_chunk(e, k)) = hi;
+          *reinterpret_cast<uint4 *>(sm + kVTL + sw64_chunk(e, k)) = lo;
         }
       }
-      mma_commit(bar_mma);
-    }
-    if (!wait_mma()) { abort = true; break; }
-    // ---- a-4/a-6: state update (registers) and the output tile ---------------
-    {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_sync(kBarChain, 128);
+      if (e == 0 && !*x.abort) {
+        tc_fence_after();
+        const uint32_t kch = sbase + kKCH + pb * 8192, kcl = sbase + kKCL + pb * 8192;
+        const uint32_t ah = sbase + kAH + pb * 2048;
+#pragma unroll 1
+        for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
+          const uint32_t aB = sbase + (part == 1 ? kVTL : kVTH);
+          const uint32_t kB = part == 2 ? kcl : kch;
+          const uint32_t mB = ah + (part == 2 ? 4096 : 0);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t ad = sdesc_sw64(aB + ks * 32, 16, 512);
+            mma_bf16(tbase + tDS, ad, sdesc_sw128(kB + ks * 2048, 4096, 1024), idS, part > 0 || ks > 0);
+            mma_bf16(tbase + tO, ad, sdesc_sw64(mB + ks * 32, 16, 512), idO, true);
+          }
+        }
+        mma_commit(&x.bar[B_DS]);
+      }
+      // state update and output tile
+      wait_bar(x, B_DS, (uint32_t)t & 1u);
+      tc_fence_after();
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         float ds[32];
-        tmem_ld32(tlane + tDS + 32 * q4, ds);
+        tmem_ld32(tl + tDS + 32 * q4, ds);
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int c = 32 * q4 + i;
-          S[c] = eG31[c] * S[c] + decC[c] * ds[i];
+          S[c] = fac[128 + c] * S[c] + fac[256 + c] * ds[i];
         }
       }
-      float ov[32];
-      tmem_ld32(tlane + tO, ov);
-      tmem_ld_wait();
-      const int e = tid;
-      __nv_bfloat16 *o = p.o + ((size_t)bh * T + t0) * D + e;
+      {
+        float ov[32];
+        tmem_ld32(tl + tO, ov);
+        tmem_ld_wait();
+        __nv_bfloat16 *o = p.o + ((size_t)bh * T + t0) * D + e;
 #pragma unroll
-      for (int r = 0; r < C; ++r)
-        if (t0 + r < T) o[(size_t)r * D] = __float2bfloat16_rn(p.scale * ov[r]);
+        for (int r = 0; r < C; ++r)
+          if (t0 + r < T) o[(size_t)r * D] = __float2bfloat16_rn(p.scale * ov[r]);
+      }
+      tc_fence_before();
+      const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
+      if (e == 0) mbar_arrive(&x.bar[B_CD0 + pb]);
+      if (!go) break;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    if (*x.abort == 0 && p.hT) {
+      float *hT = p.hT + (size_t)bh * D * D;
+#pragma unroll
+      for (int c = 0; c < D; ++c) hT[c * D + e] = S[c];
+    }
+  } else {
+    // ======================= token warpgroup =======================
+    const int tt = tid - 128;
+    const uint32_t tl = tbase + ((uint32_t)(32 * (warp - 4)) << 16);
+    const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
+    const uint32_t idG = idesc_bf16(128, 32, false, false, false);
+    const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
+    auto tma_qkg = [&](int t) {
+      mbar_arrive_expect_tx(&x.bar[B_QKG], 6 * 4096);
+      const int y = t * C;
+      tma_load_3d(sm + kRawQK, &mq, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d(sm + kRawQK + 4096, &mq, &x.bar[B_QKG], 64, y, bh);
+      tma_load_3d(sm + kRawQK + 8192, &mk, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d(sm + kRawQK + 12288, &mk, &x.bar[B_QKG], 64, y, bh);
+      tma_load_3d(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
+    };
+    auto tma_v = [&](int t) {
+      mbar_arrive_expect_tx(&x.bar[B_V], 2 * 4096);
+      tma_load_3d(sm + kRawV, &mv, &x.bar[B_V], 0, t * C, bh);
+      tma_load_3d(sm + kRawV + 4096, &mv, &x.bar[B_V], 64, t * C, bh);
+    };
+    // The solve never writes the upper off-diagonal blocks of N but its
+    // 16x16 products read them: they must hold zeros.
+    {
+      float *N = reinterpret_cast<float *>(sm + kNf);
+      for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
+      named_sync(kBarTok, 128);
+    }
+    // TMA copies issued and not yet waited for (the abort path lets them land).
+    int qkg_issued = -1, v_issued = -1;
+    if (tt == 0 && nchunks > 0) {
+      prefetch_tmap(&mq);
+      prefetch_tmap(&mk);
+      prefetch_tmap(&mv);
+      prefetch_tmap(&mg);
+      tma_qkg(0);
+      tma_v(0);
+      qkg_issued = v_issued = 0;
+    }
+    for (int t = 0; t < nchunks; ++t) {
+      const int pb = t & 1, t0 = t * C;
+      if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);
+      const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
+      token_decay(x, tt, pb, t0, T, beta);
+      fence_proxy_async_smem();
+      named_sync(kBarTok, 128);
+      if (tt == 0 && landed && !*x.abort) {
+        tc_fence_after();
+        const uint32_t qkh = sbase + kQKH + pb * 16384;
+#pragma unroll 1
+        for (int part = 0; part < 3; ++part) {  // hi*hi, lo*hi, hi*lo
+          const uint32_t aB = part == 1 ? sbase + kQKL : qkh;
+          const uint32_t bB = sbase + (part == 2 ? kKCL : kKCH) + pb * 8192;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tbase + tG, sdesc_sw128(aB + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                     sdesc_sw128(bB + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024), idG, part > 0 || ks > 0);
+        }
+        mma_commit(&x.bar[B_GRAM]);
+        if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
+          tma_qkg(t + 1);
+          qkg_issued = t + 1;
+        }
+      }
+      // A (hi/lo) and L from the Gram tile
+      wait_bar(x, B_GRAM, (uint32_t)t & 1u);
+      tc_fence_after();
+      if (warp == 4 || warp == 5) {
+        float a[32];
+        tmem_ld32(tl + tG, a);
+        tmem_ld_wait();
+        const int r = lane;
+        if (warp == 4) {
+          unsigned char *ah = sm + kAH + pb * 2048;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint4 hi, lo;
+            float m[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m[i] = (8 * k + i <= r) ? a[8 * k + i] : 0.f;
+            hi.x = split2(m[0], m[1], lo.x);
+            hi.y = split2(m[2], m[3], lo.y);
+            hi.z = split2(m[4], m[5], lo.z);
+            hi.w = split2(m[6], m[7], lo.w);
+            *reinterpret_cast<uint4 *>(ah + sw64_chunk(r, k)) = hi;
+            *reinterpret_cast<uint4 *>(ah + 4096 + sw64_chunk(r, k)) = lo;
+          }
+        } else {
+          const float br = reinterpret_cast<const float *>(sm + kBeta)[r];
+          float *L = reinterpret_cast<float *>(sm + kLf);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) L[r * 33 + j] = (j < r) ? br * a[j] : 0.f;
+        }
+      }
+      tc_fence_before();
+      named_sync(kBarTok, 128);
+      token_solve(x, tt);
+      fence_proxy_async_smem();
+      named_sync(kBarTok, 128);
+      if (tt == 0 && !*x.abort) {
+        if (wait_bar(x, B_V, (uint32_t)t & 1u)) {
+          tc_fence_after();
+          const uint32_t qkh = sbase + kQKH + pb * 16384;
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t bd = sdesc_sw64(sbase + kTT + ks * 32, 16, 512);
+            mma_bf16(tbase + tU0 + 32 * pb, sdesc_sw128(sbase + kRawV + ks * 2048, 4096, 1024), bd, idMK, ks > 0);
+            mma_bf16(tbase + tW, sdesc_sw128(qkh + 4096 + ks * 2048, 8192, 1024), bd, idMK, ks > 0);
+          }
+          mma_commit(&x.bar[B_UW]);
+        }
+      }
+      // W~ from TMEM: thread tt = key channel c writes row c of W~ stored [c][r]
+      const bool uw = wait_bar(x, B_UW, (uint32_t)t & 1u);
+      tc_fence_after();
+      if (tt == 0 && uw && t + 1 < nchunks) {  // the U MMA has consumed v
+        tma_v(t + 1);
+        v_issued = t + 1;
+      }
+      {
+        float w[32];
+        tmem_ld32(tl + tW, w);
+        tmem_ld_wait();
+        unsigned char *wt = sm + kWT + pb * 8192;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 q;
+          q.x = pack_bf16x2(w[8 * k + 0], w[8 * k + 1]);
+          q.y = pack_bf16x2(w[8 * k + 2], w[8 * k + 3]);
+          q.z = pack_bf16x2(w[8 * k + 4], w[8 * k + 5]);
+          q.w = pack_bf16x2(w[8 * k + 6], w[8 * k + 7]);
+          *reinterpret_cast<uint4 *>(wt + sw64_chunk(tt, k)) = q;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      const bool go = named_sync_and(kBarTok, 128, *x.abort == 0);
+      if (tt == 0) mbar_arrive(&x.bar[B_WT0 + pb]);
+      if (!go) break;
+    }
+    if (tt == 0 && *x.abort) {  // let every TMA already issued land before the CTA exits
+      if (qkg_issued >= 0)
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_QKG], (uint32_t)qkg_issued & 1u); ++i) {
+        }
+      if (v_issued >= 0)
+        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_V], (uint32_t)v_issued & 1u); ++i) {
+        }
+    }
   }
 
-  if (abort) {
-    if (tid == 0) {
-      atomicExch(p.status, kDevTimeout);
-      // let every TMA still in flight land before the CTA exits (bounded)
-      for (int u = tma_waited; u < tma_issued; ++u) mbar_wait(&bar_tma[u & 1], (uint32_t)(u >> 1) & 1u, kWaitLimit);
-    }
-  } else if (p.hT) {
-    float *hT = p.hT + (size_t)bh * D * D;
-#pragma unroll
-    for (int c = 0; c < D; ++c) hT[c * D + tid] = S[c];
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+  if (warp == 4) {
+    __syncwarp();
+    tmem_dealloc(tbase, kTmemCols);
+  }
 }
 
 }  // namespace

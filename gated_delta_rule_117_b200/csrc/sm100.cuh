@@ -49,6 +49,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
   return false;
 }
 
+// ---- named barriers (a subset of the CTA's warps) --------------------------------
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Barrier over `nthreads` threads that also returns the AND of `pred` over them.
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ---- async-proxy fences -------------------------------------------------------
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor core) before a barrier that releases their consumers.
@@ -132,6 +150,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t start, uint32_t lbo, ui
   return d;
 }
 
+// Same, 64-byte swizzle (rows of 64 B, 512-byte atoms of 8 rows).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)4u << 61;  // SWIZZLE_64B
+  return d;
+}
+
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          bool accumulate) {
   asm volatile(
@@ -158,6 +187,15 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t co
 // Byte offset of the 16-byte chunk `chunk` (8 bf16) of row `row`.
 __host__ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t chunk) {
   return row * 128u + (((chunk ^ row) & 7u) << 4);
+}
+
+// 64-byte swizzle: rows of 64 B (32 bf16); the 16-byte chunk index (2 bits)
+// is XORed with address bits 7-8, i.e. with (row / 2) mod 4.
+__host__ __device__ __forceinline__ uint32_t sw64_off(uint32_t row, uint32_t col) {
+  return row * 64u + ((((col >> 3) ^ (row >> 1)) & 3u) << 4) + ((col & 7u) << 1);
+}
+__host__ __device__ __forceinline__ uint32_t sw64_chunk(uint32_t row, uint32_t chunk) {
+  return row * 64u + (((chunk ^ (row >> 1)) & 3u) << 4);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -16,8 +16,10 @@ pytestmark = pytest.mark.gpu
 
 def _run(x, chunk_size=0, use_h0=True, scale=0.0, **kw):
     d = to_dev(x)
-    return kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"] if use_h0 else None,
-                         chunk_size=chunk_size, scale=scale, **kw)
+    out = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"] if use_h0 else None,
+                        chunk_size=chunk_size, scale=scale, **kw)
+    assert kda.kda_get_device_status() == 0  # no bounded wait gave up
+    return out
 
 
 def test_tiny_f32_workload():
