@@ -74,9 +74,9 @@ kda_status_t plan_prefill(int B, int H, int T, int dk, int dv, kda_dtype_t dtype
   const bool tc = chunk_size == 32 || (chunk_size == 0 && tc_ok);
   p.path = tc ? KDA_PATH_TC32 : KDA_PATH_SIMT16;
   p.chunk_size = tc ? 32 : 16;
-  p.segments = 1;
-  p.launches = (B * H == 0) ? 0 : 1;
-  p.workspace = 0;
+  p.segments = tc ? kda::tc32_segments(B * H, T) : 1;
+  p.launches = (B * H == 0) ? 0 : (p.segments > 1 ? 3 : 1);
+  p.workspace = tc ? kda::tc32_workspace(B * H, T) : 0;
   *plan = p;
   return KDA_OK;
 }
@@ -160,6 +160,8 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
   a.bf16 = dtype == KDA_DTYPE_BF16;
   a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
   a.status = kda::device_status_ptr();
+  a.workspace = workspace;
+  a.segments = plan.segments;
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
   const cudaError_t ce = plan.path == KDA_PATH_TC32 ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)

@@ -102,7 +102,18 @@ enum {
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t tG = 0, tU0 = 32, tW = 96, tO = 128, tDS = 256;
+constexpr uint32_t tG = 0, tU0 = 32, tW = 96, tO0 = 128, tDS = 256;  // tU and tO double (+32)
+
+// Launch modes.  kModeChain: one CTA per (b, h) chain over all T tokens.
+// In-device context parallelism (the report's section 5.1.1 SM-level CP,
+// composed with the segment decomposition of Eq. 17) splits every chain into
+// nseg segments of seg_len tokens:
+//   kModeSegTransition: for each segment but the last, two CTAs: one runs the
+//     segment from S = 0 (its state S~), one from S = I with v = 0 (its
+//     transition M, since the segment maps S to S~ + M S); no outputs;
+//   kModeSegFinal: one CTA per segment, entering state read from `sin`
+//     (composed by the scan kernel), writes o and, for the last segment, h_T.
+enum { kModeChain = 0, kModeSegTransition = 1, kModeSegFinal = 2 };
 
 struct TcParams {
   const __nv_bfloat16 *beta;
@@ -110,7 +121,13 @@ struct TcParams {
   __nv_bfloat16 *o;
   float *hT;
   unsigned *status;
+  const float *sin;  // [BH][nseg][128][128] entering states (kModeSegFinal)
+  float *m_out;      // [BH][nseg-1][128][128] segment transitions (kModeSegTransition)
+  float *st_out;     // [BH][nseg-1][128][128] segment states from zero (kModeSegTransition)
   int T;
+  int seg_len;
+  int nseg;
+  int mode;
   float scale;
 };
 
@@ -135,27 +152,36 @@ __device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity
 
 // hi/lo pair of (a, b): returns packed hi, writes packed lo.
 __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
-  const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
-  lo = pack_bf16x2(a - __bfloat162float(ha), b - __bfloat162float(hb));
-  __nv_bfloat162 h;
-  h.x = ha;
-  h.y = hb;
-  return *reinterpret_cast<uint32_t *>(&h);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // ---- token stage: one chunk, 128 threads (tt = 0..127) ------------------------
-__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int t0, int T, const __nv_bfloat16 *beta) {
+// Thread tt owns the key-channel pair (2pp, 2pp+1) for 16 tokens (half hf of
+// the chunk).  All shared-memory reads are staged into registers before the
+// first store so the loads are not serialised behind possibly-aliasing stores.
+__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
   unsigned char *sm = x.sm;
-  const int pp = tt & 63, hf = tt >> 6;  // channel pair (2pp, 2pp+1), token half
+  const int pp = tt & 63, hf = tt >> 6;
   const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
+  uint32_t graw[16], qraw[16], kraw[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t off = h * 4096 + sw128_off(16 * hf + i, cc);
+    graw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawG + off);
+    qraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + off);
+    kraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + 8192 + off);
+  }
   float xs0[16], xs1[16];
   float G0 = 0.f, G1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int s = 16 * hf + i;
-    const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawG + h * 4096 + sw128_off(s, cc));
-    G0 += __bfloat162float(g2.x);
-    G1 += __bfloat162float(g2.y);
+    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&graw[i]));
+    G0 += g.x;
+    G1 += g.y;
     xs0[i] = G0;
     xs1[i] = G1;
   }
@@ -167,36 +193,31 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int t0,
       xs0[i] -= G0;
       xs1[i] -= G1;
     }
-    xch[c0] = G0;
-    xch[c0 + 1] = G1;
+    *reinterpret_cast<float2 *>(xch + c0) = make_float2(G0, G1);
   } else {
     // tokens 16..31: x = sum_{16..s} g (<= 0); the half's total is G_31 - rho
-    xch[128 + c0] = G0;
-    xch[128 + c0 + 1] = G1;
+    *reinterpret_cast<float2 *>(xch + 128 + c0) = make_float2(G0, G1);
   }
-  unsigned char *qkh = sm + kQKH + p * 16384;
-  unsigned char *kch = sm + kKCH + p * 8192, *kcl = sm + kKCL + p * 8192;
+  unsigned char *qkh = sm + kQKH + p * 16384 + h * 8192;
+  unsigned char *qkl = sm + kQKL + h * 8192;
+  unsigned char *kch = sm + kKCH + p * 8192 + h * 4096, *kcl = sm + kKCL + p * 8192 + h * 4096;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int s = 16 * hf + i;
+    const uint32_t off = sw128_off(16 * hf + i, cc);
     const float x0 = fminf(fmaxf(xs0[i], -87.f), 87.f), x1 = fminf(fmaxf(xs1[i], -87.f), 87.f);
     const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
-    const uint32_t off = sw128_off(s, cc);
-    const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawQK + h * 4096 + off);
-    const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + kRawQK + 8192 + h * 4096 + off);
-    const float q0 = __bfloat162float(q2.x), q1 = __bfloat162float(q2.y);
-    const float k0 = __bfloat162float(k2.x), k1 = __bfloat162float(k2.y);
-    uint32_t lo;
-    *reinterpret_cast<uint32_t *>(qkh + h * 8192 + off) = split2(q0 * e0, q1 * e1, lo);
-    *reinterpret_cast<uint32_t *>(sm + kQKL + h * 8192 + off) = lo;
-    *reinterpret_cast<uint32_t *>(qkh + h * 8192 + 4096 + off) = split2(k0 * e0, k1 * e1, lo);
-    *reinterpret_cast<uint32_t *>(sm + kQKL + h * 8192 + 4096 + off) = lo;
-    *reinterpret_cast<uint32_t *>(kch + h * 4096 + off) = split2(k0 * i0, k1 * i1, lo);
-    *reinterpret_cast<uint32_t *>(kcl + h * 4096 + off) = lo;
-  }
-  if (tt < C) {
-    float *bet = reinterpret_cast<float *>(sm + kBeta);
-    bet[tt] = (t0 + tt < T) ? __bfloat162float(beta[t0 + tt]) : 0.f;
+    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qraw[i]));
+    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kraw[i]));
+    uint32_t qlo, klo, clo;
+    const uint32_t qhi = split2(q.x * e0, q.y * e1, qlo);
+    const __nv_bfloat162 khi = __floats2bfloat162_rn(k.x * e0, k.y * e1);
+    const uint32_t chi = split2(k.x * i0, k.y * i1, clo);
+    (void)klo;
+    *reinterpret_cast<uint32_t *>(qkh + off) = qhi;
+    *reinterpret_cast<__nv_bfloat162 *>(qkh + 4096 + off) = khi;
+    *reinterpret_cast<uint32_t *>(qkl + off) = qlo;
+    *reinterpret_cast<uint32_t *>(kch + off) = chi;
+    *reinterpret_cast<uint32_t *>(kcl + off) = clo;
   }
   named_sync(kBarTok, 128);
   {
@@ -283,12 +304,34 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
   }
 }
 
+// Row e of S~^T = (Diag(e^rho) S)^T for the 32 channels [32 q, 32 q + 32):
+// four 16-byte chunks of bf16 in the SW128 K-major layout of the S~^T operand.
+__device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const float *__restrict__ erho,
+                                           const float (&S)[D], int e, int q) {
+  float4 r[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = reinterpret_cast<const float4 *>(erho + 32 * q)[i];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = 32 * q + 8 * k;
+    const float4 a = r[2 * k], b = r[2 * k + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x * S[c + 0], a.y * S[c + 1]);
+    w.y = pack_bf16x2(a.z * S[c + 2], a.w * S[c + 3]);
+    w.z = pack_bf16x2(b.x * S[c + 4], b.y * S[c + 5]);
+    w.w = pack_bf16x2(b.z * S[c + 6], b.w * S[c + 7]);
+    *reinterpret_cast<uint4 *>(st + (q >> 1) * 16384 + sw128_chunk(e, (q & 1) * 4 + k)) = w;
+  }
+}
+
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
                     const TcParams p) {
-  extern __shared__ unsigned char smraw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) unsigned char smraw[];
+  // 1024-byte aligned base, derived by pointer arithmetic so that every access
+  // through it stays a shared-memory (not generic) access.
+  unsigned char *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
   Ctx x;
   x.sm = sm;
   x.bar = reinterpret_cast<uint64_t *>(sm + kBar);
@@ -297,9 +340,35 @@ __global__ void __launch_bounds__(NT, 1)
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
   const int T = p.T;
-  const int nchunks = (T + C - 1) / C;
+  // which chain, which token range, where the entering and final states live
+  int bh = blockIdx.x, seg = 0, kind = 0;  // kind 1: state from zero, 2: transition
+  if (p.mode == kModeSegTransition) {
+    const int per = 2 * (p.nseg - 1);
+    bh = blockIdx.x / per;
+    seg = (blockIdx.x % per) >> 1;
+    kind = 1 + (blockIdx.x & 1);
+  } else if (p.mode == kModeSegFinal) {
+    bh = blockIdx.x / p.nseg;
+    seg = blockIdx.x % p.nseg;
+  }
+  const int tb = seg * p.seg_len;
+  const int te = min(T, tb + p.seg_len);
+  const int nchunks = (te - tb + C - 1) / C;
+  const bool v_zero = kind == 2;
+  const bool store_o = p.mode != kModeSegTransition;
+  const float *h0src = nullptr;
+  float *hdst = nullptr;
+  if (p.mode == kModeChain) {
+    h0src = p.h0 ? p.h0 + (size_t)bh * D * D : nullptr;
+    hdst = p.hT ? p.hT + (size_t)bh * D * D : nullptr;
+  } else if (p.mode == kModeSegTransition) {
+    const size_t slot = ((size_t)bh * (p.nseg - 1) + seg) * D * D;
+    hdst = (kind == 1 ? p.st_out : p.m_out) + slot;
+  } else {
+    h0src = p.sin + ((size_t)bh * p.nseg + seg) * D * D;
+    hdst = (seg == p.nseg - 1 && p.hT) ? p.hT + (size_t)bh * D * D : nullptr;
+  }
   const uint32_t sbase = smem_u32(sm);
 
   if (tid == 0) {
@@ -323,43 +392,38 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t idV = idesc_bf16(128, 32, false, true, true);   // -S~^T W~^T (B MN-major)
     const uint32_t idO = idesc_bf16(128, 32, false, false, false);
     const uint32_t idS = idesc_bf16(128, 128, false, true, false);
+    unsigned char *st = sm + kST;
     float S[D];
-    {
-      const float *h0 = p.h0 ? p.h0 + (size_t)bh * D * D : nullptr;
 #pragma unroll
-      for (int c = 0; c < D; ++c) S[c] = h0 ? h0[c * D + e] : 0.f;
-    }
-    for (int t = 0; t < nchunks; ++t) {
-      const int pb = t & 1, t0 = t * C;
-      const bool ready = wait_bar(x, B_WT0 + pb, (uint32_t)(t >> 1) & 1u);
-      const float *fac = reinterpret_cast<const float *>(sm + kFac + pb * 1536);
-      // S~^T(t): row e, c-blocks 0/1, eight 16-byte chunks each
+    for (int c = 0; c < D; ++c) S[c] = h0src ? h0src[c * D + e] : (kind == 2 && c == e ? 1.f : 0.f);
+    // V~(t) -= S~^T W~^T onto U(t), and O(t) = S~^T Qs^T; called by all of warp 0.
+    auto issue_v1 = [&](int t) {
+      const int pb = t & 1;
+      tc_fence_after();
+      const uint64_t dS = sdesc_sw128(sbase + kST, 16, 1024);
+      const uint64_t dW = sdesc_sw64(sbase + kWT + pb * 8192, 8192, 512);
+      const uint64_t dQ = sdesc_sw128(sbase + kQKH + pb * 16384, 16, 1024);
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t ad = sdesc_add(dS, (ks >> 2) * 16384 + (ks & 3) * 32);
+        mma_bf16_warp(tbase + tU0 + 32 * pb, ad, sdesc_add(dW, ks * 1024), idV, true);
+        mma_bf16_warp(tbase + tO0 + 32 * pb, ad, sdesc_add(dQ, (ks >> 2) * 8192 + (ks & 3) * 32), idO, ks > 0);
+      }
+      mma_commit_warp(&x.bar[B_V1]);
+    };
+    if (nchunks > 0) {
+      const bool ready = wait_bar(x, B_WT0, 0u);
+      const float *erho = reinterpret_cast<const float *>(sm + kFac);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c0 = h * 64 + k * 8;
-          uint4 w;
-          w.x = pack_bf16x2(fac[c0 + 0] * S[c0 + 0], fac[c0 + 1] * S[c0 + 1]);
-          w.y = pack_bf16x2(fac[c0 + 2] * S[c0 + 2], fac[c0 + 3] * S[c0 + 3]);
-          w.z = pack_bf16x2(fac[c0 + 4] * S[c0 + 4], fac[c0 + 5] * S[c0 + 5]);
-          w.w = pack_bf16x2(fac[c0 + 6] * S[c0 + 6], fac[c0 + 7] * S[c0 + 7]);
-          *reinterpret_cast<uint4 *>(sm + kST + h * 16384 + sw128_chunk(e, k)) = w;
-        }
+      for (int q = 0; q < 4; ++q) store_st32(st, erho, S, e, q);
       fence_proxy_async_smem();
       tc_fence_before();
       named_sync(kBarChain, 128);
-      if (e == 0 && ready && !*x.abort) {
-        tc_fence_after();
-        const uint32_t st = sbase + kST, wt = sbase + kWT + pb * 8192, qkh = sbase + kQKH + pb * 16384;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t ad = sdesc_sw128(st + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tbase + tU0 + 32 * pb, ad, sdesc_sw64(wt + ks * 1024, 8192, 512), idV, true);
-          mma_bf16(tbase + tO, ad, sdesc_sw128(qkh + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), idO, ks > 0);
-        }
-        mma_commit(&x.bar[B_V1]);
-      }
+      if (warp == 0 && __shfl_sync(0xffffffffu, ready && !*x.abort, 0)) issue_v1(0);
+    }
+    for (int t = 0; t < nchunks; ++t) {
+      const int pb = t & 1, t0 = tb + t * C;
+      const bool has_next = t + 1 < nchunks;
       // V~^T(t) -> bf16 hi/lo operands
       wait_bar(x, B_V1, (uint32_t)t & 1u);
       tc_fence_after();
@@ -381,56 +445,76 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       named_sync(kBarChain, 128);
-      if (e == 0 && !*x.abort) {
+      if (warp == 0 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
         tc_fence_after();
-        const uint32_t kch = sbase + kKCH + pb * 8192, kcl = sbase + kKCL + pb * 8192;
-        const uint32_t ah = sbase + kAH + pb * 2048;
-#pragma unroll 1
+        const uint64_t dVh = sdesc_sw64(sbase + kVTH, 16, 512), dVl = sdesc_sw64(sbase + kVTL, 16, 512);
+        const uint64_t dKh = sdesc_sw128(sbase + kKCH + pb * 8192, 4096, 1024);
+        const uint64_t dKl = sdesc_sw128(sbase + kKCL + pb * 8192, 4096, 1024);
+        const uint64_t dAh = sdesc_sw64(sbase + kAH + pb * 2048, 16, 512), dAl = sdesc_add(dAh, 4096);
+#pragma unroll
         for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
-          const uint32_t aB = sbase + (part == 1 ? kVTL : kVTH);
-          const uint32_t kB = part == 2 ? kcl : kch;
-          const uint32_t mB = ah + (part == 2 ? 4096 : 0);
+          const uint64_t aB = part == 1 ? dVl : dVh;
+          const uint64_t kB = part == 2 ? dKl : dKh;
+          const uint64_t mB = part == 2 ? dAl : dAh;
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t ad = sdesc_sw64(aB + ks * 32, 16, 512);
-            mma_bf16(tbase + tDS, ad, sdesc_sw128(kB + ks * 2048, 4096, 1024), idS, part > 0 || ks > 0);
-            mma_bf16(tbase + tO, ad, sdesc_sw64(mB + ks * 32, 16, 512), idO, true);
+            const uint64_t ad = sdesc_add(aB, ks * 32);
+            mma_bf16_warp(tbase + tDS, ad, sdesc_add(kB, ks * 2048), idS, part > 0 || ks > 0);
+            mma_bf16_warp(tbase + tO0 + 32 * pb, ad, sdesc_add(mB, ks * 32), idO, true);
           }
         }
-        mma_commit(&x.bar[B_DS]);
+        mma_commit_warp(&x.bar[B_DS]);
       }
-      // state update and output tile
+      // the next chunk's factors are needed to write S~^T(t+1) in the update pass
+      bool next_ready = true;
+      if (has_next) next_ready = wait_bar(x, B_WT0 + (pb ^ 1), (uint32_t)((t + 1) >> 1) & 1u);
       wait_bar(x, B_DS, (uint32_t)t & 1u);
       tc_fence_after();
+      {
+        const float *fac = reinterpret_cast<const float *>(sm + kFac + pb * 1536);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float ds[32];
-        tmem_ld32(tl + tDS + 32 * q4, ds);
-        tmem_ld_wait();
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float ds[32];
+          tmem_ld32(tl + tDS + 32 * q4, ds);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = 32 * q4 + i;
-          S[c] = fac[128 + c] * S[c] + fac[256 + c] * ds[i];
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 a = reinterpret_cast<const float4 *>(fac + 128 + 32 * q4)[i4];
+            const float4 b = reinterpret_cast<const float4 *>(fac + 256 + 32 * q4)[i4];
+            const int c = 32 * q4 + 4 * i4;
+            S[c + 0] = a.x * S[c + 0] + b.x * ds[4 * i4 + 0];
+            S[c + 1] = a.y * S[c + 1] + b.y * ds[4 * i4 + 1];
+            S[c + 2] = a.z * S[c + 2] + b.z * ds[4 * i4 + 2];
+            S[c + 3] = a.w * S[c + 3] + b.w * ds[4 * i4 + 3];
+          }
         }
       }
-      {
+      if (has_next) {
+        const float *erho = reinterpret_cast<const float *>(sm + kFac + (pb ^ 1) * 1536);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) store_st32(st, erho, S, e, q);
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
+      if (e == 0) mbar_arrive(&x.bar[B_CD0 + pb]);  // chunk t's buffers are free for chunk t + 2
+      if (warp == 0 && __shfl_sync(0xffffffffu, has_next && next_ready && go, 0)) issue_v1(t + 1);
+      // output tile of chunk t (its TMEM half is not touched by chunk t + 1)
+      if (store_o) {
         float ov[32];
-        tmem_ld32(tl + tO, ov);
+        tmem_ld32(tl + tO0 + 32 * pb, ov);
         tmem_ld_wait();
         __nv_bfloat16 *o = p.o + ((size_t)bh * T + t0) * D + e;
 #pragma unroll
         for (int r = 0; r < C; ++r)
-          if (t0 + r < T) o[(size_t)r * D] = __float2bfloat16_rn(p.scale * ov[r]);
+          if (t0 + r < te) o[(size_t)r * D] = __float2bfloat16_rn(p.scale * ov[r]);
       }
       tc_fence_before();
-      const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
-      if (e == 0) mbar_arrive(&x.bar[B_CD0 + pb]);
       if (!go) break;
     }
-    if (*x.abort == 0 && p.hT) {
-      float *hT = p.hT + (size_t)bh * D * D;
+    if (*x.abort == 0 && hdst) {
 #pragma unroll
-      for (int c = 0; c < D; ++c) hT[c * D + e] = S[c];
+      for (int c = 0; c < D; ++c) hdst[c * D + e] = S[c];
     }
   } else {
     // ======================= token warpgroup =======================
@@ -439,59 +523,83 @@ __global__ void __launch_bounds__(NT, 1)
     const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
     const uint32_t idG = idesc_bf16(128, 32, false, false, false);
     const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
+    // TMA issue, called by all of warp 4 (one elected lane issues).
     auto tma_qkg = [&](int t) {
-      mbar_arrive_expect_tx(&x.bar[B_QKG], 6 * 4096);
-      const int y = t * C;
-      tma_load_3d(sm + kRawQK, &mq, &x.bar[B_QKG], 0, y, bh);
-      tma_load_3d(sm + kRawQK + 4096, &mq, &x.bar[B_QKG], 64, y, bh);
-      tma_load_3d(sm + kRawQK + 8192, &mk, &x.bar[B_QKG], 0, y, bh);
-      tma_load_3d(sm + kRawQK + 12288, &mk, &x.bar[B_QKG], 64, y, bh);
-      tma_load_3d(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
-      tma_load_3d(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
+      mbar_arrive_expect_tx_warp(&x.bar[B_QKG], 6 * 4096);
+      const int y = tb + t * C;
+      tma_load_3d_warp(sm + kRawQK, &mq, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d_warp(sm + kRawQK + 4096, &mq, &x.bar[B_QKG], 64, y, bh);
+      tma_load_3d_warp(sm + kRawQK + 8192, &mk, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d_warp(sm + kRawQK + 12288, &mk, &x.bar[B_QKG], 64, y, bh);
+      tma_load_3d_warp(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
+      tma_load_3d_warp(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
     };
     auto tma_v = [&](int t) {
-      mbar_arrive_expect_tx(&x.bar[B_V], 2 * 4096);
-      tma_load_3d(sm + kRawV, &mv, &x.bar[B_V], 0, t * C, bh);
-      tma_load_3d(sm + kRawV + 4096, &mv, &x.bar[B_V], 64, t * C, bh);
+      if (v_zero) return;  // transition runs: v = 0, the buffer holds zeros
+      mbar_arrive_expect_tx_warp(&x.bar[B_V], 2 * 4096);
+      tma_load_3d_warp(sm + kRawV, &mv, &x.bar[B_V], 0, tb + t * C, bh);
+      tma_load_3d_warp(sm + kRawV + 4096, &mv, &x.bar[B_V], 64, tb + t * C, bh);
     };
     // The solve never writes the upper off-diagonal blocks of N but its
     // 16x16 products read them: they must hold zeros.
     {
       float *N = reinterpret_cast<float *>(sm + kNf);
       for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
+      // Ks lo is not kept (its rounding is negligible for L): the Gram's lo
+      // pass reads these quarters of QKL, which therefore hold zeros.
+      uint4 *z0 = reinterpret_cast<uint4 *>(sm + kQKL + 4096), *z1 = reinterpret_cast<uint4 *>(sm + kQKL + 12288);
+      for (int i = tt; i < 256; i += 128) {
+        z0[i] = make_uint4(0, 0, 0, 0);
+        z1[i] = make_uint4(0, 0, 0, 0);
+      }
+      if (v_zero) {  // v = 0 for a transition run: the U MMA then yields U = 0
+        uint4 *zv = reinterpret_cast<uint4 *>(sm + kRawV);
+        for (int i = tt; i < 512; i += 128) zv[i] = make_uint4(0, 0, 0, 0);
+      }
       named_sync(kBarTok, 128);
     }
     // TMA copies issued and not yet waited for (the abort path lets them land).
     int qkg_issued = -1, v_issued = -1;
-    if (tt == 0 && nchunks > 0) {
-      prefetch_tmap(&mq);
-      prefetch_tmap(&mk);
-      prefetch_tmap(&mv);
-      prefetch_tmap(&mg);
+    if (warp == 4 && nchunks > 0) {
+      if (lane == 0) {
+        prefetch_tmap(&mq);
+        prefetch_tmap(&mk);
+        prefetch_tmap(&mv);
+        prefetch_tmap(&mg);
+      }
       tma_qkg(0);
       tma_v(0);
-      qkg_issued = v_issued = 0;
+      qkg_issued = 0;
+      v_issued = v_zero ? -1 : 0;
     }
+    // beta goes through shared memory one chunk ahead: the global load for
+    // chunk t + 1 is issued at the top of chunk t and stored at its end.
+    float *bet = reinterpret_cast<float *>(sm + kBeta);
+    if (tt < C) bet[tt] = (tb + tt < te) ? __bfloat162float(beta[tb + tt]) : 0.f;
     for (int t = 0; t < nchunks; ++t) {
-      const int pb = t & 1, t0 = t * C;
+      const int pb = t & 1, t0 = tb + t * C;
+      float beta_next = 0.f;
+      if (tt < C && t0 + C + tt < te) beta_next = __bfloat162float(beta[t0 + C + tt]);
       if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);
       const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
-      token_decay(x, tt, pb, t0, T, beta);
+      token_decay(x, tt, pb);
       fence_proxy_async_smem();
       named_sync(kBarTok, 128);
-      if (tt == 0 && landed && !*x.abort) {
+      if (warp == 4 && __shfl_sync(0xffffffffu, landed && !*x.abort, 0)) {
         tc_fence_after();
-        const uint32_t qkh = sbase + kQKH + pb * 16384;
-#pragma unroll 1
+        const uint64_t dQh = sdesc_sw128(sbase + kQKH + pb * 16384, 16, 1024), dQl = sdesc_sw128(sbase + kQKL, 16, 1024);
+        const uint64_t dKh = sdesc_sw128(sbase + kKCH + pb * 8192, 16, 1024);
+        const uint64_t dKl = sdesc_sw128(sbase + kKCL + pb * 8192, 16, 1024);
+#pragma unroll
         for (int part = 0; part < 3; ++part) {  // hi*hi, lo*hi, hi*lo
-          const uint32_t aB = part == 1 ? sbase + kQKL : qkh;
-          const uint32_t bB = sbase + (part == 2 ? kKCL : kKCH) + pb * 8192;
+          const uint64_t aB = part == 1 ? dQl : dQh;
+          const uint64_t bB = part == 2 ? dKl : dKh;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tbase + tG, sdesc_sw128(aB + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                     sdesc_sw128(bB + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024), idG, part > 0 || ks > 0);
+            mma_bf16_warp(tbase + tG, sdesc_add(aB, (ks >> 2) * 8192 + (ks & 3) * 32),
+                          sdesc_add(bB, (ks >> 2) * 4096 + (ks & 3) * 32), idG, part > 0 || ks > 0);
         }
-        mma_commit(&x.bar[B_GRAM]);
+        mma_commit_warp(&x.bar[B_GRAM]);
         if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
           tma_qkg(t + 1);
           qkg_issued = t + 1;
@@ -532,25 +640,28 @@ __global__ void __launch_bounds__(NT, 1)
       token_solve(x, tt);
       fence_proxy_async_smem();
       named_sync(kBarTok, 128);
-      if (tt == 0 && !*x.abort) {
-        if (wait_bar(x, B_V, (uint32_t)t & 1u)) {
+      if (warp == 4 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
+        const bool vok = v_zero || wait_bar(x, B_V, (uint32_t)t & 1u);
+        if (__shfl_sync(0xffffffffu, vok, 0)) {
           tc_fence_after();
-          const uint32_t qkh = sbase + kQKH + pb * 16384;
+          const uint64_t dT = sdesc_sw64(sbase + kTT, 16, 512);
+          const uint64_t dV = sdesc_sw128(sbase + kRawV, 4096, 1024);
+          const uint64_t dKs = sdesc_sw128(sbase + kQKH + pb * 16384 + 4096, 8192, 1024);
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t bd = sdesc_sw64(sbase + kTT + ks * 32, 16, 512);
-            mma_bf16(tbase + tU0 + 32 * pb, sdesc_sw128(sbase + kRawV + ks * 2048, 4096, 1024), bd, idMK, ks > 0);
-            mma_bf16(tbase + tW, sdesc_sw128(qkh + 4096 + ks * 2048, 8192, 1024), bd, idMK, ks > 0);
+            const uint64_t bd = sdesc_add(dT, ks * 32);
+            mma_bf16_warp(tbase + tU0 + 32 * pb, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
+            mma_bf16_warp(tbase + tW, sdesc_add(dKs, ks * 2048), bd, idMK, ks > 0);
           }
-          mma_commit(&x.bar[B_UW]);
+          mma_commit_warp(&x.bar[B_UW]);
         }
       }
       // W~ from TMEM: thread tt = key channel c writes row c of W~ stored [c][r]
       const bool uw = wait_bar(x, B_UW, (uint32_t)t & 1u);
       tc_fence_after();
-      if (tt == 0 && uw && t + 1 < nchunks) {  // the U MMA has consumed v
+      if (warp == 4 && __shfl_sync(0xffffffffu, uw, 0) && t + 1 < nchunks) {  // the U MMA has consumed v
         tma_v(t + 1);
-        v_issued = t + 1;
+        if (!v_zero) v_issued = t + 1;
       }
       {
         float w[32];
@@ -567,13 +678,14 @@ __global__ void __launch_bounds__(NT, 1)
           *reinterpret_cast<uint4 *>(wt + sw64_chunk(tt, k)) = q;
         }
       }
+      if (tt < C) bet[tt] = beta_next;  // the solve of chunk t has read beta(t)
       fence_proxy_async_smem();
       tc_fence_before();
       const bool go = named_sync_and(kBarTok, 128, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_WT0 + pb]);
       if (!go) break;
     }
-    if (tt == 0 && *x.abort) {  // let every TMA already issued land before the CTA exits
+    if (tt == 0 && *x.abort) {  // let every TMA already issued land before the CTA exits (warp 4 issued them)
       if (qkg_issued >= 0)
         for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_QKG], (uint32_t)qkg_issued & 1u); ++i) {
         }
@@ -592,12 +704,85 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
+// Entering states of the segments, column block by column block:
+// S_in(0) = h0 (or 0); S_in(s+1) = M_s S_in(s) + S~_s  (Eq. 17's prefix scan).
+// Grid (B*H, 8): each CTA owns 16 state columns of one chain; fp32 throughout.
+__global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const float *M, const float *St, float *Sin,
+                                                      int nseg) {
+  extern __shared__ float cps[];
+  float *Ms = cps;               // [128][129]
+  float *X = cps + 128 * 129;    // [128][16]
+  const int bh = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
+  const int i = tid >> 1, j0 = 8 * (tid & 1);
+  const size_t mat = (size_t)D * D;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = h0 ? h0[bh * mat + (size_t)i * D + c0 + j0 + j] : 0.f;
+  for (int s = 0;; ++s) {
+    float *out = Sin + ((size_t)bh * nseg + s) * mat + (size_t)i * D + c0 + j0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      out[j] = acc[j];
+      X[i * 16 + j0 + j] = acc[j];
+    }
+    if (s + 1 >= nseg) break;
+    const float *Mg = M + ((size_t)bh * (nseg - 1) + s) * mat;
+    for (int e = tid; e < D * D / 4; e += 256) {
+      const float4 m4 = reinterpret_cast<const float4 *>(Mg)[e];
+      const int r = (4 * e) / D, c = (4 * e) % D;
+      Ms[r * 129 + c] = m4.x;
+      Ms[r * 129 + c + 1] = m4.y;
+      Ms[r * 129 + c + 2] = m4.z;
+      Ms[r * 129 + c + 3] = m4.w;
+    }
+    __syncthreads();
+    const float *Sg = St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = Sg[j];
+    for (int k = 0; k < D; ++k) {
+      const float m = Ms[i * 129 + k];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += m * X[k * 16 + j0 + j];
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
+
+void tc32_plan(int BH, int T, int *segments, int *seg_len) {
+  // Fill the 148 SMs (one CTA each) when there are few chains; segments of at
+  // least 256 tokens keep the extra passes worthwhile.  Segment lengths are
+  // whole chunks; the count is recomputed so no segment is empty.
+  *segments = 1;
+  *seg_len = T > 0 ? T : 1;
+  if (BH <= 0 || BH > 74 || T <= 0) return;
+  const int by_sm = 148 / BH, by_len = T / 256;
+  const int p0 = by_sm < by_len ? by_sm : by_len;
+  if (p0 <= 1) return;
+  const int len = ((T + p0 - 1) / p0 + C - 1) / C * C;
+  *seg_len = len;
+  *segments = (T + len - 1) / len;
+}
+
+int tc32_segments(int BH, int T) {
+  int P, L;
+  tc32_plan(BH, T, &P, &L);
+  return P;
+}
+
+size_t tc32_workspace(int BH, int T) {
+  const int P = tc32_segments(BH, T);
+  if (P <= 1) return 0;
+  const size_t mat = (size_t)D * D * sizeof(float);
+  return (size_t)BH * (2 * (P - 1) + P) * mat;
+}
 
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   if (a.B * a.H == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, mg;
-  const uint64_t T = (uint64_t)(a.T > 0 ? a.T : 1), n = (uint64_t)a.B * a.H;
+  const int BH = a.B * a.H;
+  const uint64_t T = (uint64_t)(a.T > 0 ? a.T : 1), n = (uint64_t)BH;
   if (!encode_tmap_bf16_3d(&mq, a.q, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mk, a.k, D, T, n, 64, C) ||
       !encode_tmap_bf16_3d(&mv, a.v, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mg, a.g, D, T, n, 64, C))
     return cudaErrorInvalidValue;
@@ -607,11 +792,41 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.o = (__nv_bfloat16 *)a.o;
   p.hT = a.hT;
   p.status = a.status;
+  p.sin = nullptr;
+  p.m_out = p.st_out = nullptr;
   p.T = a.T;
   p.scale = a.scale;
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  chunk_tc_kernel<<<a.B * a.H, NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+  const int P = a.segments > 1 ? a.segments : 1;
+  if (P == 1) {
+    p.seg_len = a.T > 0 ? a.T : 1;
+    p.nseg = 1;
+    p.mode = kModeChain;
+    chunk_tc_kernel<<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+    return cudaGetLastError();
+  }
+  const size_t mat = (size_t)D * D;
+  float *ws = static_cast<float *>(a.workspace);
+  float *Mw = ws, *Sw = ws + (size_t)BH * (P - 1) * mat, *Sin = Sw + (size_t)BH * (P - 1) * mat;
+  int P2, L;
+  tc32_plan(BH, a.T, &P2, &L);
+  if (P2 != P) return cudaErrorInvalidValue;
+  p.seg_len = L;
+  p.nseg = P;
+  p.m_out = Mw;
+  p.st_out = Sw;
+  p.sin = Sin;
+  p.mode = kModeSegTransition;
+  chunk_tc_kernel<<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int scan_smem = (128 * 129 + 128 * 16) * (int)sizeof(float);
+  if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
+    return e;
+  cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, P);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  p.mode = kModeSegFinal;
+  chunk_tc_kernel<<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
   return cudaGetLastError();
 }
 

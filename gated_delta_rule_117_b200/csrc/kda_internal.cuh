@@ -22,6 +22,8 @@ struct ChunkArgs {
   int bf16;     // 1: q,k,v,g,beta,o are bf16; 0: fp32
   float scale;  // resolved (> 0)
   unsigned *status;
+  void *workspace;  // scratch of at least the planned size (context-parallel passes)
+  int segments;     // in-device context-parallel segments per chain (1 = none)
 };
 
 struct DecodeArgs {
@@ -35,6 +37,10 @@ struct DecodeArgs {
 
 cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t s);
+// Planning of the tensor-core path: segments per chain, segment length, workspace bytes.
+void tc32_plan(int BH, int T, int *segments, int *seg_len);
+int tc32_segments(int BH, int T);
+size_t tc32_workspace(int BH, int T);
 cudaError_t launch_recurrent_step(const DecodeArgs &a, cudaStream_t s);
 
 }  // namespace kda

@@ -66,6 +66,41 @@ def test_fast_decay_heads_both_paths():
         assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"], chunk
 
 
+@pytest.mark.parametrize("B,H,T", [(1, 16, 2305), (1, 2, 2304), (2, 3, 1100), (1, 74, 600)])
+def test_in_device_context_parallel(B, H, T):
+    # few chains and enough tokens: the call splits every chain into segments
+    # (transition pass, scan, final pass); results must match the recurrence
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=B, H=H, T=T, seed=123)
+    plan = kda.kda_chunk_fwd_plan(B, H, T, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    assert plan["segments"] > 1 and plan["launches"] == 3 and plan["workspace"] > 0
+    x = synth.prefill_inputs(w)
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_context_parallel_inplace_state_and_missing_workspace():
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=8, T=1024, seed=5)
+    x = synth.prefill_inputs(w)
+    d = to_dev(x)
+    assert kda.kda_chunk_fwd_plan(1, 8, 1024, 128, 128, kda.KDA_DTYPE_BF16, 0)["segments"] > 1
+    o_ref, h_ref = oracle_prefill(x)
+    h = d["h0"].clone()
+    o, _ = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h, h_T=h)
+    assert kda.kda_get_device_status() == 0
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(h, h_ref) <= TOL["bf16"]
+    ws = kda.kda_chunk_fwd_workspace_size(1, 8, 1024, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    st = kda.kda_chunk_fwd(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["g"].data_ptr(),
+                           d["beta"].data_ptr(), None, o.data_ptr(), None, 1, 8, 1024, 128, 128,
+                           kda.KDA_DTYPE_BF16, 0, 0.0, None, 0, None)
+    assert st == 6  # KDA_ERR_WORKSPACE
+    small = torch.empty(ws - 16, dtype=torch.uint8, device="cuda")
+    st = kda.kda_chunk_fwd(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["g"].data_ptr(),
+                           d["beta"].data_ptr(), None, o.data_ptr(), None, 1, 8, 1024, 128, 128,
+                           kda.KDA_DTYPE_BF16, 0, 0.0, small.data_ptr(), small.numel(), None)
+    assert st == 6
+
+
 def test_prefill_workload_reduced_T():
     w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=700)
     x = synth.prefill_inputs(w)
