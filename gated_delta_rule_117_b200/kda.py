@@ -23,7 +23,8 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
                 "KDA_ERR_ALIAS", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT",
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
-            "kda_status_string", "kda_get_device_status", "kda_version"]
+            "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
+            "kda_noalloc_scratch_bytes"]
 
 
 class KdaError(RuntimeError):
@@ -66,6 +67,10 @@ def load_library():
             lib.kda_get_device_status.restype = i
             lib.kda_version.argtypes = []
             lib.kda_version.restype = i
+            lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 8 + [i] * 7 + [f, vp]
+            lib.kda_chunk_fwd_noalloc.restype = i
+            lib.kda_noalloc_scratch_bytes.argtypes = []
+            lib.kda_noalloc_scratch_bytes.restype = sz
             _lib = lib
     return _lib
 
@@ -98,6 +103,17 @@ def kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_si
     """Returns the raw kda_status_t."""
     return load_library().kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size,
                                         scale, workspace, workspace_bytes, stream)
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
+    """kda_chunk_fwd with libkda's own fixed scratch array (no workspace argument).
+    For callers that cannot allocate device memory.  Returns the raw kda_status_t."""
+    return load_library().kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size,
+                                                scale, stream)
+
+
+def kda_noalloc_scratch_bytes() -> int:
+    return load_library().kda_noalloc_scratch_bytes()
 
 
 def kda_recurrent_step(q, k, v, g, beta, S, o, B, H, dk, dv, dtype, scale, stream) -> int:

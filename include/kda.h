@@ -141,6 +141,33 @@ kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, con
                                 const void *beta, float *S, void *o, int B, int H, int dk, int dv,
                                 kda_dtype_t dtype, float scale, kda_stream_t stream);
 
+/*
+ * Prefill without a caller-provided workspace, for callers that cannot
+ * allocate device memory (e.g. a plugin inside a host framework that owns the
+ * GPU memory pool and exposes no allocator, or a latency-critical path where
+ * cudaMalloc's possible device synchronisation is not acceptable).  The
+ * source report has no counterpart to this entry point: it is a packaging
+ * variant of kda_chunk_fwd.
+ *
+ * Same arguments, layouts, alignment and aliasing rules and results as
+ * kda_chunk_fwd, minus workspace/workspace_bytes: the scratch comes from one
+ * fixed device array inside libkda of kda_noalloc_scratch_bytes() bytes
+ * (32 MiB), held on every GPU that loads the library until the process exits.
+ * Returns KDA_ERR_WORKSPACE if the call would need more scratch than that.
+ * The first call on a device (with that device current) looks up the array's
+ * device address once (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  No call allocates or frees memory.  All calls share the
+ * array and nothing in it needs to start at zero; calls that overlap on the
+ * GPU (different streams or host threads) race on it, so serialise them.
+ */
+kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
+                                   const void *beta, const float *h0, void *o, float *h_T, int B,
+                                   int H, int T, int dk, int dv, kda_dtype_t dtype, int chunk_size,
+                                   float scale, kda_stream_t stream);
+
+/* Size in bytes of the fixed scratch array kda_chunk_fwd_noalloc uses. */
+size_t kda_noalloc_scratch_bytes(void);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(kda_status_t s);
 
