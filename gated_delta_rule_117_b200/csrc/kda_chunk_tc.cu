@@ -18,14 +18,16 @@
 //     S' = Diag(e^{G_31}) S + Diag(e^{G_31 - rho}) Kc^T V~
 // Every tensor-core product is issued "transposed" so that M = 128 is a
 // channel dimension and the TMEM lane is the channel an epilogue thread owns:
-//     Gram  D[r|32+r][j] = [Qs; Ks] Kc^T          (M = 128: rows 64..127 unused)
+//     Gram  D[.][j|32+j] = [Ks; Qs_lo; Qs; -] [Kc_hi | Kc_lo]^T   (one N = 64 product;
+//           A = Qs Kc_hi + Qs Kc_lo + Qs_lo Kc_hi,  L = Ks Kc_hi + Ks Kc_lo)
 //     U^T   D[e][r]      = V^T T^T,   W~^T D[c][r] = Ks^T T^T
-//     V~^T  D[e][r]     -= S~^T W~^T               (negated A, accumulated onto U^T)
-//     O^T   D[e][r]      = S~^T Qs^T + V~^T A^T
+//     [O^T | V~^T] D     = S~^T [Qs; -W~]^T + [0 | U^T]          (one N = 64 product)
+//     O^T   D[e][r]     += V~^T A^T
 //     dS^T  D[e][c]      = V~^T Kc
 // Qs and Kc (Gram), A and V~ (output), V~ and Kc (state update) enter as
-// hi + lo bf16 pairs multiplied as hi*hi + lo*hi + hi*lo; without that their
-// bf16 rounding would dominate the error.
+// hi + lo bf16 pairs (hi*hi + lo*hi + hi*lo); without that their bf16
+// rounding would dominate the error.  MMAs are few and wide on purpose: each
+// tcgen05.mma carries a fixed cost that dominates small-N products.
 //
 // Work split (the report's token-parallel stage vs head-parallel recurrence,
 // section 5.1.1, mapped onto one CTA per (b, h) chain), 8 warps:
@@ -65,25 +67,23 @@ constexpr uint32_t kBarChain = 1, kBarTok = 2;
 constexpr int kRawQK = 0;        // q h0 | q h1 | k h0 | k h1 (TMA)
 constexpr int kRawG = 16384;     // g h0 | g h1 (TMA)
 constexpr int kRawV = 24576;     // v h0 | v h1 (TMA; the U MMA reads it in place)
-constexpr int kQKH = 32768;      // [2]: Qs hi h0 | Ks hi h0 | Qs hi h1 | Ks hi h1
-constexpr int kQKL = 65536;      // Qs lo / Ks lo, same layout (Gram only)
-constexpr int kKCH = 81920;      // [2]: Kc hi h0 | h1
-constexpr int kKCL = 98304;      // [2]: Kc lo h0 | h1
-constexpr int kST = 114688;      // S~^T [e][c], K-halves of 16 KB (SW128)
-constexpr int kVTH = 147456;     // V~^T hi [e][j] (SW64, 64-byte rows)
-constexpr int kVTL = 155648;     // V~^T lo
-constexpr int kWT = 163840;      // [2]: W~ stored [c][r] (SW64), 8 KB each
-constexpr int kAH = 180224;      // [2]: A hi [r][j] (SW64), 2 KB each; A lo at +4096
+constexpr int kQKW = 32768;      // [2] x 32 KB; per channel block (16 KB): Ks | Qs lo | Qs | -W~, 4 KB each
+constexpr int kKC = 98304;       // [2] x 16 KB; per channel block (8 KB): Kc hi | Kc lo
+constexpr int kST = 131072;      // S~^T [e][c], K-halves of 16 KB (SW128)
+constexpr int kVTH = 163840;     // V~^T hi [e][j] (SW64, 64-byte rows)
+constexpr int kVTL = 172032;     // V~^T lo
+constexpr int kAH = 180224;      // [2] x 4 KB: A hi [r][j] (SW64) | A lo
 constexpr int kTT = 188416;      // T [r][s] (SW64)
 constexpr int kLf = 190464;      // fp32 L [32][33]
 constexpr int kNf = 194688;      // fp32 N = (I + L)^-1 [32][33]
 constexpr int kXf = 198912;      // fp32 scratch [16][17]
-constexpr int kFac = 200000;     // [2]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
-constexpr int kXch = 203072;     // fp32 rho[128], G_31 - rho[128]
-constexpr int kBeta = 204096;    // fp32 beta[32]
-constexpr int kBar = 204224;     // mbarriers
-constexpr int kMisc = 204480;    // TMEM base address, abort flag
-constexpr int kSmemBytes = 204496 + 1024;
+constexpr int kXa = 200000;      // fp32 [32][33]: Qs_lo Kc_hi part of A
+constexpr int kFac = 204224;     // [2]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
+constexpr int kXch = 207296;     // fp32 rho[128], G_31 - rho[128]
+constexpr int kBeta = 208320;    // fp32 beta[32]
+constexpr int kBar = 208448;     // mbarriers
+constexpr int kMisc = 208704;    // TMEM base address, abort flag
+constexpr int kSmemBytes = 208720 + 1024;
 
 // barrier slots
 enum {
@@ -100,9 +100,10 @@ enum {
   B_COUNT
 };
 
-// TMEM columns (fp32, 128 lanes)
+// TMEM columns (fp32, 128 lanes).  The output and pseudo-value accumulators
+// of a chunk parity are adjacent ([O | U]) so one N = 64 MMA updates both.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t tG = 0, tU0 = 32, tW = 96, tO0 = 128, tDS = 256;  // tU and tO double (+32)
+constexpr uint32_t tG = 0, tOU = 64, tW = 192, tDS = 256;  // tO(p) = tOU + 64 p, tU(p) = tO(p) + 32
 
 // Launch modes.  kModeChain: one CTA per (b, h) chain over all T tokens.
 // In-device context parallelism (the report's section 5.1.1 SM-level CP,
@@ -138,12 +139,16 @@ struct Ctx {
   unsigned *status;
 };
 
-// Bounded wait that also returns (false) as soon as another role aborted.
+// Bounded wait: sleeps on the barrier (no spinning), returns false as soon as
+// another role aborted, and gives up after 2 s of wall time.
 __device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity) {
   uint64_t *b = &x.bar[slot];
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
+  if (mbar_try_wait(b, parity)) return true;
+  const uint64_t t_start = global_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(b, parity, 1000000u)) return true;
     if (*x.abort) return false;
+    if (global_ns() - t_start > 2000000000ull) break;
   }
   *x.abort = 1;
   atomicExch(x.status, kDevTimeout);
@@ -198,9 +203,8 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
     // tokens 16..31: x = sum_{16..s} g (<= 0); the half's total is G_31 - rho
     *reinterpret_cast<float2 *>(xch + 128 + c0) = make_float2(G0, G1);
   }
-  unsigned char *qkh = sm + kQKH + p * 16384 + h * 8192;
-  unsigned char *qkl = sm + kQKL + h * 8192;
-  unsigned char *kch = sm + kKCH + p * 8192 + h * 4096, *kcl = sm + kKCL + p * 8192 + h * 4096;
+  unsigned char *qkw = sm + kQKW + p * 32768 + h * 16384;  // Ks | Qs lo | Qs | -W~
+  unsigned char *kc = sm + kKC + p * 16384 + h * 8192;     // Kc hi | Kc lo
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint32_t off = sw128_off(16 * hf + i, cc);
@@ -208,16 +212,15 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
     const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
     const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qraw[i]));
     const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kraw[i]));
-    uint32_t qlo, klo, clo;
+    uint32_t qlo, clo;
     const uint32_t qhi = split2(q.x * e0, q.y * e1, qlo);
     const __nv_bfloat162 khi = __floats2bfloat162_rn(k.x * e0, k.y * e1);
     const uint32_t chi = split2(k.x * i0, k.y * i1, clo);
-    (void)klo;
-    *reinterpret_cast<uint32_t *>(qkh + off) = qhi;
-    *reinterpret_cast<__nv_bfloat162 *>(qkh + 4096 + off) = khi;
-    *reinterpret_cast<uint32_t *>(qkl + off) = qlo;
-    *reinterpret_cast<uint32_t *>(kch + off) = chi;
-    *reinterpret_cast<uint32_t *>(kcl + off) = clo;
+    *reinterpret_cast<__nv_bfloat162 *>(qkw + off) = khi;
+    *reinterpret_cast<uint32_t *>(qkw + 4096 + off) = qlo;
+    *reinterpret_cast<uint32_t *>(qkw + 8192 + off) = qhi;
+    *reinterpret_cast<uint32_t *>(kc + off) = chi;
+    *reinterpret_cast<uint32_t *>(kc + 4096 + off) = clo;
   }
   named_sync(kBarTok, 128);
   {
@@ -389,25 +392,27 @@ __global__ void __launch_bounds__(NT, 1)
     // ======================= chain warpgroup =======================
     const int e = tid;
     const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
-    const uint32_t idV = idesc_bf16(128, 32, false, true, true);   // -S~^T W~^T (B MN-major)
     const uint32_t idO = idesc_bf16(128, 32, false, false, false);
+    const uint32_t idOU = idesc_bf16(128, 64, false, false, false);
     const uint32_t idS = idesc_bf16(128, 128, false, true, false);
     unsigned char *st = sm + kST;
     float S[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) S[c] = h0src ? h0src[c * D + e] : (kind == 2 && c == e ? 1.f : 0.f);
-    // V~(t) -= S~^T W~^T onto U(t), and O(t) = S~^T Qs^T; called by all of warp 0.
+    // [O(t) | V~(t)] = S~^T [Qs; -W~]^T + [0 | U(t)]; called by all of warp 0.  The
+    // first K-step is split so O starts from zero while V~ accumulates onto U.
     auto issue_v1 = [&](int t) {
       const int pb = t & 1;
       tc_fence_after();
       const uint64_t dS = sdesc_sw128(sbase + kST, 16, 1024);
-      const uint64_t dW = sdesc_sw64(sbase + kWT + pb * 8192, 8192, 512);
-      const uint64_t dQ = sdesc_sw128(sbase + kQKH + pb * 16384, 16, 1024);
+      const uint64_t dB = sdesc_sw128(sbase + kQKW + pb * 32768 + 8192, 16, 1024);  // rows: Qs, -W~
+      const uint32_t tO = tbase + tOU + 64 * pb;
+      mma_bf16_warp(tO, dS, dB, idO, false);
+      mma_bf16_warp(tO + 32, dS, sdesc_add(dB, 4096), idO, true);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = sdesc_add(dS, (ks >> 2) * 16384 + (ks & 3) * 32);
-        mma_bf16_warp(tbase + tU0 + 32 * pb, ad, sdesc_add(dW, ks * 1024), idV, true);
-        mma_bf16_warp(tbase + tO0 + 32 * pb, ad, sdesc_add(dQ, (ks >> 2) * 8192 + (ks & 3) * 32), idO, ks > 0);
+      for (int ks = 1; ks < 8; ++ks) {
+        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+        mma_bf16_warp(tO, sdesc_add(dS, koff), sdesc_add(dB, koff), idOU, true);
       }
       mma_commit_warp(&x.bar[B_V1]);
     };
@@ -429,7 +434,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       {
         float v[32];
-        tmem_ld32(tl + tU0 + 32 * pb, v);
+        tmem_ld32(tl + tOU + 64 * pb + 32, v);
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -448,9 +453,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (warp == 0 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
         tc_fence_after();
         const uint64_t dVh = sdesc_sw64(sbase + kVTH, 16, 512), dVl = sdesc_sw64(sbase + kVTL, 16, 512);
-        const uint64_t dKh = sdesc_sw128(sbase + kKCH + pb * 8192, 4096, 1024);
-        const uint64_t dKl = sdesc_sw128(sbase + kKCL + pb * 8192, 4096, 1024);
-        const uint64_t dAh = sdesc_sw64(sbase + kAH + pb * 2048, 16, 512), dAl = sdesc_add(dAh, 4096);
+        const uint64_t dKh = sdesc_sw128(sbase + kKC + pb * 16384, 8192, 1024), dKl = sdesc_add(dKh, 4096);
+        const uint64_t dAh = sdesc_sw64(sbase + kAH + pb * 4096, 16, 512), dAl = sdesc_add(dAh, 2048);
 #pragma unroll
         for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
           const uint64_t aB = part == 1 ? dVl : dVh;
@@ -460,7 +464,7 @@ __global__ void __launch_bounds__(NT, 1)
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = sdesc_add(aB, ks * 32);
             mma_bf16_warp(tbase + tDS, ad, sdesc_add(kB, ks * 2048), idS, part > 0 || ks > 0);
-            mma_bf16_warp(tbase + tO0 + 32 * pb, ad, sdesc_add(mB, ks * 32), idO, true);
+            mma_bf16_warp(tbase + tOU + 64 * pb, ad, sdesc_add(mB, ks * 32), idO, true);
           }
         }
         mma_commit_warp(&x.bar[B_DS]);
@@ -502,7 +506,7 @@ __global__ void __launch_bounds__(NT, 1)
       // output tile of chunk t (its TMEM half is not touched by chunk t + 1)
       if (store_o) {
         float ov[32];
-        tmem_ld32(tl + tO0 + 32 * pb, ov);
+        tmem_ld32(tl + tOU + 64 * pb, ov);
         tmem_ld_wait();
         __nv_bfloat16 *o = p.o + ((size_t)bh * T + t0) * D + e;
 #pragma unroll
@@ -521,7 +525,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int tt = tid - 128;
     const uint32_t tl = tbase + ((uint32_t)(32 * (warp - 4)) << 16);
     const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
-    const uint32_t idG = idesc_bf16(128, 32, false, false, false);
+    const uint32_t idG = idesc_bf16(128, 64, false, false, false);
     const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
     // TMA issue, called by all of warp 4 (one elected lane issues).
     auto tma_qkg = [&](int t) {
@@ -545,13 +549,6 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float *N = reinterpret_cast<float *>(sm + kNf);
       for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
-      // Ks lo is not kept (its rounding is negligible for L): the Gram's lo
-      // pass reads these quarters of QKL, which therefore hold zeros.
-      uint4 *z0 = reinterpret_cast<uint4 *>(sm + kQKL + 4096), *z1 = reinterpret_cast<uint4 *>(sm + kQKL + 12288);
-      for (int i = tt; i < 256; i += 128) {
-        z0[i] = make_uint4(0, 0, 0, 0);
-        z1[i] = make_uint4(0, 0, 0, 0);
-      }
       if (v_zero) {  // v = 0 for a transition run: the U MMA then yields U = 0
         uint4 *zv = reinterpret_cast<uint4 *>(sm + kRawV);
         for (int i = tt; i < 512; i += 128) zv[i] = make_uint4(0, 0, 0, 0);
@@ -587,56 +584,65 @@ __global__ void __launch_bounds__(NT, 1)
       named_sync(kBarTok, 128);
       if (warp == 4 && __shfl_sync(0xffffffffu, landed && !*x.abort, 0)) {
         tc_fence_after();
-        const uint64_t dQh = sdesc_sw128(sbase + kQKH + pb * 16384, 16, 1024), dQl = sdesc_sw128(sbase + kQKL, 16, 1024);
-        const uint64_t dKh = sdesc_sw128(sbase + kKCH + pb * 8192, 16, 1024);
-        const uint64_t dKl = sdesc_sw128(sbase + kKCL + pb * 8192, 16, 1024);
+        // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
+        const uint64_t dA = sdesc_sw128(sbase + kQKW + pb * 32768, 16, 1024);
+        const uint64_t dB = sdesc_sw128(sbase + kKC + pb * 16384, 16, 1024);
 #pragma unroll
-        for (int part = 0; part < 3; ++part) {  // hi*hi, lo*hi, hi*lo
-          const uint64_t aB = part == 1 ? dQl : dQh;
-          const uint64_t bB = part == 2 ? dKl : dKh;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_bf16_warp(tbase + tG, sdesc_add(aB, (ks >> 2) * 8192 + (ks & 3) * 32),
-                          sdesc_add(bB, (ks >> 2) * 4096 + (ks & 3) * 32), idG, part > 0 || ks > 0);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_warp(tbase + tG, sdesc_add(dA, (ks >> 2) * 16384 + (ks & 3) * 32),
+                        sdesc_add(dB, (ks >> 2) * 8192 + (ks & 3) * 32), idG, ks > 0);
         mma_commit_warp(&x.bar[B_GRAM]);
         if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
           tma_qkg(t + 1);
           qkg_issued = t + 1;
         }
       }
-      // A (hi/lo) and L from the Gram tile
+      // L (lanes 0-31, Ks rows) and A (lanes 64-95, Qs rows, plus the Qs lo
+      // part from lanes 32-63) from the Gram tile
       wait_bar(x, B_GRAM, (uint32_t)t & 1u);
       tc_fence_after();
-      if (warp == 4 || warp == 5) {
-        float a[32];
+      float a[32];
+      if (warp == 4 || warp == 6) {
+        float b[32];
         tmem_ld32(tl + tG, a);
+        tmem_ld32(tl + tG + 32, b);
         tmem_ld_wait();
-        const int r = lane;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a[j] += b[j];
         if (warp == 4) {
-          unsigned char *ah = sm + kAH + pb * 2048;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint4 hi, lo;
-            float m[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m[i] = (8 * k + i <= r) ? a[8 * k + i] : 0.f;
-            hi.x = split2(m[0], m[1], lo.x);
-            hi.y = split2(m[2], m[3], lo.y);
-            hi.z = split2(m[4], m[5], lo.z);
-            hi.w = split2(m[6], m[7], lo.w);
-            *reinterpret_cast<uint4 *>(ah + sw64_chunk(r, k)) = hi;
-            *reinterpret_cast<uint4 *>(ah + 4096 + sw64_chunk(r, k)) = lo;
-          }
-        } else {
+          const int r = lane;
           const float br = reinterpret_cast<const float *>(sm + kBeta)[r];
           float *L = reinterpret_cast<float *>(sm + kLf);
 #pragma unroll
           for (int j = 0; j < 32; ++j) L[r * 33 + j] = (j < r) ? br * a[j] : 0.f;
         }
+      } else if (warp == 5) {
+        tmem_ld32(tl + tG, a);
+        tmem_ld_wait();
+        float *Xa = reinterpret_cast<float *>(sm + kXa);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) Xa[lane * 33 + j] = a[j];
       }
       tc_fence_before();
       named_sync(kBarTok, 128);
+      if (warp == 6) {
+        const int r = lane;
+        const float *Xa = reinterpret_cast<const float *>(sm + kXa);
+        unsigned char *ah = sm + kAH + pb * 4096;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 hi, lo;
+          float m[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m[i] = (8 * k + i <= r) ? a[8 * k + i] + Xa[r * 33 + 8 * k + i] : 0.f;
+          hi.x = split2(m[0], m[1], lo.x);
+          hi.y = split2(m[2], m[3], lo.y);
+          hi.z = split2(m[4], m[5], lo.z);
+          hi.w = split2(m[6], m[7], lo.w);
+          *reinterpret_cast<uint4 *>(ah + sw64_chunk(r, k)) = hi;
+          *reinterpret_cast<uint4 *>(ah + 2048 + sw64_chunk(r, k)) = lo;
+        }
+      }
       token_solve(x, tt);
       fence_proxy_async_smem();
       named_sync(kBarTok, 128);
@@ -646,11 +652,11 @@ __global__ void __launch_bounds__(NT, 1)
           tc_fence_after();
           const uint64_t dT = sdesc_sw64(sbase + kTT, 16, 512);
           const uint64_t dV = sdesc_sw128(sbase + kRawV, 4096, 1024);
-          const uint64_t dKs = sdesc_sw128(sbase + kQKH + pb * 16384 + 4096, 8192, 1024);
+          const uint64_t dKs = sdesc_sw128(sbase + kQKW + pb * 32768, 16384, 1024);
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t bd = sdesc_add(dT, ks * 32);
-            mma_bf16_warp(tbase + tU0 + 32 * pb, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
+            mma_bf16_warp(tbase + tOU + 64 * pb + 32, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
             mma_bf16_warp(tbase + tW, sdesc_add(dKs, ks * 2048), bd, idMK, ks > 0);
           }
           mma_commit_warp(&x.bar[B_UW]);
@@ -664,19 +670,15 @@ __global__ void __launch_bounds__(NT, 1)
         if (!v_zero) v_issued = t + 1;
       }
       {
+        // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand block
         float w[32];
         tmem_ld32(tl + tW, w);
         tmem_ld_wait();
-        unsigned char *wt = sm + kWT + pb * 8192;
+        const int c = tt, h = c >> 6, cc = c & 63;
+        unsigned char *nw = sm + kQKW + pb * 32768 + h * 16384 + 12288;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint4 q;
-          q.x = pack_bf16x2(w[8 * k + 0], w[8 * k + 1]);
-          q.y = pack_bf16x2(w[8 * k + 2], w[8 * k + 3]);
-          q.z = pack_bf16x2(w[8 * k + 4], w[8 * k + 5]);
-          q.w = pack_bf16x2(w[8 * k + 6], w[8 * k + 7]);
-          *reinterpret_cast<uint4 *>(wt + sw64_chunk(tt, k)) = q;
-        }
+        for (int r = 0; r < C; ++r)
+          *reinterpret_cast<__nv_bfloat16 *>(nw + sw128_off(r, cc)) = __float2bfloat16_rn(-w[r]);
       }
       if (tt < C) bet[tt] = beta_next;  // the solve of chunk t has read beta(t)
       fence_proxy_async_smem();
