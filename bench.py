@@ -112,6 +112,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def rank_workload(w, rank):
+    """Weak scaling: every rank runs its own replica of the workload on its own
+    seeded inputs (the (b, h) chains are independent; nothing is exchanged)."""
+    return w if rank == 0 else w.with_(seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(value, dist=None, device=None):
+    """Max of a per-rank scalar over all ranks (the job's time is the slowest rank's)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, max_ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def gpu_uuid(torch, dev):
     u = str(torch.cuda.get_device_properties(dev).uuid)
     return u if u.startswith("GPU-") else "GPU-" + u
@@ -171,6 +192,7 @@ def main():
         print(json.dumps(measure_decode(args, synth, kda, torch, dev, pk, pk_kind)))
         return
     assert not w.decode, "main line is a prefill workload"
+    w = rank_workload(w, rank)
     x = synth.prefill_inputs(w)
     d = {k: v.to(dev) for k, v in x.items()}
     h0 = d["h0"] if w.h0_std > 0 else None
@@ -210,14 +232,9 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
     times_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(times_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times_ms), dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
-    tokens = B * T * world
-    value = tokens / (ms_per_step / 1e3)
+    value = job_throughput(B * T, world, ms_per_step)
     kern_ms = statistics.mean(times_ms)  # one launch per step: the step is the kernel
     bytes_per_launch = synth.prefill_bytes(w)
     achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9

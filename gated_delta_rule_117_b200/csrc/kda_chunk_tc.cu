@@ -57,7 +57,8 @@ using namespace sm100;
 
 constexpr int C = 32;     // tokens per chunk
 constexpr int D = 128;    // dk = dv
-constexpr int NT = 256;   // 8 warps
+constexpr int NT = 384;   // 12 warps: chain warpgroup + two token warpgroups
+constexpr int NTOK = 256;  // token-stage threads
 constexpr uint32_t kWaitLimit = 1u << 22;  // polls; seconds, far beyond any real wait
 constexpr uint32_t kBarChain = 1, kBarTok = 2;
 
@@ -79,11 +80,12 @@ constexpr int kNf = 194688;      // fp32 N = (I + L)^-1 [32][33]
 constexpr int kXf = 198912;      // fp32 scratch [16][17]
 constexpr int kXa = 200000;      // fp32 [32][33]: Qs_lo Kc_hi part of A
 constexpr int kFac = 204224;     // [2]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
-constexpr int kXch = 207296;     // fp32 rho[128], G_31 - rho[128]
-constexpr int kBeta = 208320;    // fp32 beta[32]
-constexpr int kBar = 208448;     // mbarriers
-constexpr int kMisc = 208704;    // TMEM base address, abort flag
-constexpr int kSmemBytes = 208720 + 1024;
+constexpr int kXch = 207296;     // fp32 [4][128]: per-quarter sums of g (8 tokens each)
+constexpr int kBeta = 209344;    // fp32 beta[32]
+constexpr int kBar = 209472;     // mbarriers
+constexpr int kMisc = 209728;    // TMEM base address, abort flag
+constexpr int kOst = 210944;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
+constexpr int kSmemBytes = 219136 + 1024;
 
 // barrier slots
 enum {
@@ -164,51 +166,52 @@ __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// ---- token stage: one chunk, 128 threads (tt = 0..127) ------------------------
-// Thread tt owns the key-channel pair (2pp, 2pp+1) for 16 tokens (half hf of
-// the chunk).  All shared-memory reads are staged into registers before the
-// first store so the loads are not serialised behind possibly-aliasing stores.
+// ---- token stage: one chunk, 256 threads (tt = 0..255) ------------------------
+// Thread tt owns the key-channel pair (2pp, 2pp+1) for the 8 tokens of
+// quarter qt of the chunk.  The chunk-local cumulative decay is assembled from
+// the quarters' sums (exchanged through shared memory).  All shared-memory
+// reads are staged into registers before the first store so they are not
+// serialised behind possibly-aliasing stores.
 __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
   unsigned char *sm = x.sm;
-  const int pp = tt & 63, hf = tt >> 6;
+  const int pp = tt & 63, qt = tt >> 6;
   const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
-  uint32_t graw[16], qraw[16], kraw[16];
+  uint32_t graw[8], qraw[8], kraw[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t off = h * 4096 + sw128_off(16 * hf + i, cc);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t off = h * 4096 + sw128_off(8 * qt + i, cc);
     graw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawG + off);
     qraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + off);
     kraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + 8192 + off);
   }
-  float xs0[16], xs1[16];
+  float xs0[8], xs1[8];
   float G0 = 0.f, G1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&graw[i]));
     G0 += g.x;
     G1 += g.y;
     xs0[i] = G0;
     xs1[i] = G1;
   }
-  float *xch = reinterpret_cast<float *>(sm + kXch);
-  if (hf == 0) {
-    // tokens 0..15: x = G_s - G_15 (>= 0); G_15 = rho
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      xs0[i] -= G0;
-      xs1[i] -= G1;
-    }
-    *reinterpret_cast<float2 *>(xch + c0) = make_float2(G0, G1);
-  } else {
-    // tokens 16..31: x = sum_{16..s} g (<= 0); the half's total is G_31 - rho
-    *reinterpret_cast<float2 *>(xch + 128 + c0) = make_float2(G0, G1);
+  float *xq = reinterpret_cast<float *>(sm + kXch);  // [quarter][channel] sums
+  *reinterpret_cast<float2 *>(xq + 128 * qt + c0) = make_float2(G0, G1);
+  named_sync(kBarTok, NTOK);
+  // x = G_s - G_15 with G_15 = (sum of quarters 0, 1): quarter offsets
+  float o0, o1;
+  {
+    const float2 s0 = *reinterpret_cast<const float2 *>(xq + c0);
+    const float2 s1 = *reinterpret_cast<const float2 *>(xq + 128 + c0);
+    const float2 s2 = *reinterpret_cast<const float2 *>(xq + 256 + c0);
+    o0 = qt == 0 ? -(s0.x + s1.x) : qt == 1 ? -s1.x : qt == 2 ? 0.f : s2.x;
+    o1 = qt == 0 ? -(s0.y + s1.y) : qt == 1 ? -s1.y : qt == 2 ? 0.f : s2.y;
   }
   unsigned char *qkw = sm + kQKW + p * 32768 + h * 16384;  // Ks | Qs lo | Qs | -W~
   unsigned char *kc = sm + kKC + p * 16384 + h * 8192;     // Kc hi | Kc lo
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t off = sw128_off(16 * hf + i, cc);
-    const float x0 = fminf(fmaxf(xs0[i], -87.f), 87.f), x1 = fminf(fmaxf(xs1[i], -87.f), 87.f);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t off = sw128_off(8 * qt + i, cc);
+    const float x0 = fminf(fmaxf(xs0[i] + o0, -87.f), 87.f), x1 = fminf(fmaxf(xs1[i] + o1, -87.f), 87.f);
     const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
     const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qraw[i]));
     const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kraw[i]));
@@ -222,11 +225,10 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
     *reinterpret_cast<uint32_t *>(kc + off) = chi;
     *reinterpret_cast<uint32_t *>(kc + 4096 + off) = clo;
   }
-  named_sync(kBarTok, 128);
-  {
+  if (tt < 128) {
     const int c = tt;
     float *fac = reinterpret_cast<float *>(sm + kFac + p * 1536);
-    const float rho = xch[c], tail = xch[128 + c];
+    const float rho = xq[c] + xq[128 + c], tail = xq[256 + c] + xq[384 + c];
     fac[c] = __expf(rho);                // e^rho
     fac[128 + c] = __expf(rho + tail);   // e^{G_31}
     fac[256 + c] = __expf(tail);         // e^{G_31 - rho}
@@ -234,7 +236,7 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
 }
 
 // N = (I + L)^-1 for the strictly lower 32x32 L in Lf (fp32), blocked 8 -> 16 -> 32,
-// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  128 threads.
+// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  256 threads.
 __device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
   unsigned char *sm = x.sm;
   const float *L = reinterpret_cast<const float *>(sm + kLf);
@@ -254,56 +256,54 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
       N[(b0 + r) * 33 + b0 + jj] = acc;
     }
   }
-  named_sync(kBarTok, 128);
+  named_sync(kBarTok, NTOK);
   // level 2: N_10 = -N_11 L_10 N_00 inside each 16x16 block (8x8 pieces)
-  {
+  if (tt < 128) {
     const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) acc += L[(o + 8 + r) * 33 + o + s] * N[(o + s) * 33 + o + j];
     X[blk * 64 + e] = acc;
   }
-  named_sync(kBarTok, 128);
-  {
+  named_sync(kBarTok, NTOK);
+  if (tt < 128) {
     const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) acc += N[(o + 8 + r) * 33 + o + 8 + s] * X[blk * 64 + s * 8 + j];
     N[(o + 8 + r) * 33 + o + j] = -acc;
   }
-  named_sync(kBarTok, 128);
-  // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (2 elements per thread)
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+  named_sync(kBarTok, NTOK);
+  // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (one element per thread)
+  {
+    const int r = tt >> 4, j = tt & 15;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += L[(16 + r) * 33 + s] * N[s * 33 + j];
     X[r * 17 + j] = acc;
   }
-  named_sync(kBarTok, 128);
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+  named_sync(kBarTok, NTOK);
+  {
+    const int r = tt >> 4, j = tt & 15;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += N[(16 + r) * 33 + 16 + s] * X[s * 17 + j];
     N[(16 + r) * 33 + j] = -acc;
   }
-  named_sync(kBarTok, 128);
-  // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 8-column chunk k)
+  named_sync(kBarTok, NTOK);
+  // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 4-column piece)
   {
-    const int r = tt >> 2, k = tt & 3;
-    uint4 w;
+    const int r = tt >> 3, k = (tt >> 1) & 3, half = tt & 1;
+    uint2 w;
     uint32_t *pw = &w.x;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j0 = 8 * k + 2 * i;
+    for (int i = 0; i < 2; ++i) {
+      const int j0 = 8 * k + 4 * half + 2 * i;
       const float a0 = (j0 <= r) ? N[r * 33 + j0] * bet[j0] : 0.f;
       const float a1 = (j0 + 1 <= r) ? N[r * 33 + j0 + 1] * bet[j0 + 1] : 0.f;
       pw[i] = pack_bf16x2(a0, a1);
     }
-    *reinterpret_cast<uint4 *>(sm + kTT + sw64_chunk(r, k)) = w;
+    *reinterpret_cast<uint2 *>(sm + kTT + sw64_chunk(r, k) + 8 * half) = w;
   }
 }
 
@@ -330,7 +330,7 @@ __device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
-                    const TcParams p) {
+                    const __grid_constant__ CUtensorMap mo, const TcParams p) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   // 1024-byte aligned base, derived by pointer arithmetic so that every access
   // through it stays a shared-memory (not generic) access.
@@ -390,6 +390,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   if (warp < 4) {
     // ======================= chain warpgroup =======================
+    regs_increase<248>();
     const int e = tid;
     const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
     const uint32_t idO = idesc_bf16(128, 32, false, false, false);
@@ -503,27 +504,40 @@ __global__ void __launch_bounds__(NT, 1)
       const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
       if (e == 0) mbar_arrive(&x.bar[B_CD0 + pb]);  // chunk t's buffers are free for chunk t + 2
       if (warp == 0 && __shfl_sync(0xffffffffu, has_next && next_ready && go, 0)) issue_v1(t + 1);
-      // output tile of chunk t (its TMEM half is not touched by chunk t + 1)
+      // output tile of chunk t (its TMEM half is not touched by chunk t + 1):
+      // column e goes into a swizzled shared tile that one TMA store writes out
+      // (rows past the end of the sequence are clipped by the tensor map)
       if (store_o) {
         float ov[32];
         tmem_ld32(tl + tOU + 64 * pb, ov);
         tmem_ld_wait();
-        __nv_bfloat16 *o = p.o + ((size_t)bh * T + t0) * D + e;
+        unsigned char *ot = sm + kOst + (e >> 6) * 4096;
 #pragma unroll
         for (int r = 0; r < C; ++r)
-          if (t0 + r < te) o[(size_t)r * D] = __float2bfloat16_rn(p.scale * ov[r]);
+          *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(r, e & 63)) = __float2bfloat16_rn(p.scale * ov[r]);
+        fence_proxy_async_smem();
+        named_sync(kBarChain, 128);
+        if (warp == 0) {
+          tma_store_3d_warp(&mo, sm + kOst, 0, t0, bh);
+          tma_store_3d_warp(&mo, sm + kOst + 4096, 64, t0, bh);
+          bulk_commit_warp();
+          if (lane == 0) bulk_wait_read_all();  // the tile is rewritten next chunk
+        }
       }
       tc_fence_before();
       if (!go) break;
     }
+    if (warp == 0 && lane == 0) bulk_wait_all();
     if (*x.abort == 0 && hdst) {
 #pragma unroll
       for (int c = 0; c < D; ++c) hdst[c * D + e] = S[c];
     }
   } else {
-    // ======================= token warpgroup =======================
+    // ======================= token warpgroups (8 warps) =======================
+    regs_decrease<120>();
     const int tt = tid - 128;
-    const uint32_t tl = tbase + ((uint32_t)(32 * (warp - 4)) << 16);
+    const int quarter = warp & 3, half = (warp >> 3) & 1;  // TMEM lane quarter; which half of the columns
+    const uint32_t tl = tbase + ((uint32_t)(32 * quarter) << 16);
     const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
     const uint32_t idG = idesc_bf16(128, 64, false, false, false);
     const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
@@ -548,12 +562,12 @@ __global__ void __launch_bounds__(NT, 1)
     // 16x16 products read them: they must hold zeros.
     {
       float *N = reinterpret_cast<float *>(sm + kNf);
-      for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
+      for (int i = tt; i < 32 * 33; i += NTOK) N[i] = 0.f;
       if (v_zero) {  // v = 0 for a transition run: the U MMA then yields U = 0
         uint4 *zv = reinterpret_cast<uint4 *>(sm + kRawV);
-        for (int i = tt; i < 512; i += 128) zv[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tt; i < 512; i += NTOK) zv[i] = make_uint4(0, 0, 0, 0);
       }
-      named_sync(kBarTok, 128);
+      named_sync(kBarTok, NTOK);
     }
     // TMA copies issued and not yet waited for (the abort path lets them land).
     int qkg_issued = -1, v_issued = -1;
@@ -570,18 +584,19 @@ __global__ void __launch_bounds__(NT, 1)
       v_issued = v_zero ? -1 : 0;
     }
     // beta goes through shared memory one chunk ahead: the global load for
-    // chunk t + 1 is issued at the top of chunk t and stored at its end.
+    // chunk t + 1 is issued at the top of chunk t and converted at its end.
     float *bet = reinterpret_cast<float *>(sm + kBeta);
+    const unsigned short *beta_bits = reinterpret_cast<const unsigned short *>(beta);
     if (tt < C) bet[tt] = (tb + tt < te) ? __bfloat162float(beta[tb + tt]) : 0.f;
     for (int t = 0; t < nchunks; ++t) {
       const int pb = t & 1, t0 = tb + t * C;
-      float beta_next = 0.f;
-      if (tt < C && t0 + C + tt < te) beta_next = __bfloat162float(beta[t0 + C + tt]);
+      unsigned short beta_next = 0;
+      if (tt < C && t0 + C + tt < te) beta_next = __ldg(beta_bits + t0 + C + tt);
       if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);
       const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
       token_decay(x, tt, pb);
       fence_proxy_async_smem();
-      named_sync(kBarTok, 128);
+      named_sync(kBarTok, NTOK);
       if (warp == 4 && __shfl_sync(0xffffffffu, landed && !*x.abort, 0)) {
         tc_fence_after();
         // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
@@ -597,44 +612,48 @@ __global__ void __launch_bounds__(NT, 1)
           qkg_issued = t + 1;
         }
       }
-      // L (lanes 0-31, Ks rows) and A (lanes 64-95, Qs rows, plus the Qs lo
-      // part from lanes 32-63) from the Gram tile
+      // Gram tile -> L (lanes 0-31: Ks rows) and A (lanes 64-95: Qs rows, plus
+      // the Qs-lo part from lanes 32-63); two warps per lane quarter, each
+      // taking 16 of the 32 columns j.
       wait_bar(x, B_GRAM, (uint32_t)t & 1u);
       tc_fence_after();
-      float a[32];
-      if (warp == 4 || warp == 6) {
-        float b[32];
-        tmem_ld32(tl + tG, a);
-        tmem_ld32(tl + tG + 32, b);
+      float a[16];
+      const int r = lane, j0 = 16 * half;
+      if (quarter == 0 || quarter == 2) {
+        float b[16];
+        tmem_ld16(tl + tG + j0, a);
+        tmem_ld16(tl + tG + 32 + j0, b);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) a[j] += b[j];
-        if (warp == 4) {
-          const int r = lane;
-          const float br = reinterpret_cast<const float *>(sm + kBeta)[r];
-          float *L = reinterpret_cast<float *>(sm + kLf);
+        for (int j = 0; j < 16; ++j) a[j] += b[j];
+        if (quarter == 0) {
+          const float br = bet[r];
+          float *Lm = reinterpret_cast<float *>(sm + kLf);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) L[r * 33 + j] = (j < r) ? br * a[j] : 0.f;
+          for (int j = 0; j < 16; ++j) Lm[r * 33 + j0 + j] = (j0 + j < r) ? br * a[j] : 0.f;
         }
-      } else if (warp == 5) {
-        tmem_ld32(tl + tG, a);
+      } else if (quarter == 1) {
+        tmem_ld16(tl + tG + j0, a);
         tmem_ld_wait();
         float *Xa = reinterpret_cast<float *>(sm + kXa);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) Xa[lane * 33 + j] = a[j];
+        for (int j = 0; j < 16; ++j) Xa[r * 33 + j0 + j] = a[j];
       }
       tc_fence_before();
-      named_sync(kBarTok, 128);
-      if (warp == 6) {
-        const int r = lane;
+      named_sync(kBarTok, NTOK);
+      if (quarter == 2) {
         const float *Xa = reinterpret_cast<const float *>(sm + kXa);
         unsigned char *ah = sm + kAH + pb * 4096;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int kk = 0; kk < 2; ++kk) {
+          const int k = 2 * half + kk;
           uint4 hi, lo;
           float m[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m[i] = (8 * k + i <= r) ? a[8 * k + i] + Xa[r * 33 + 8 * k + i] : 0.f;
+          for (int i = 0; i < 8; ++i) {
+            const int j = 8 * k + i;
+            m[i] = (j <= r) ? a[8 * kk + i] + Xa[r * 33 + j] : 0.f;
+          }
           hi.x = split2(m[0], m[1], lo.x);
           hi.y = split2(m[2], m[3], lo.y);
           hi.z = split2(m[4], m[5], lo.z);
@@ -645,7 +664,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       token_solve(x, tt);
       fence_proxy_async_smem();
-      named_sync(kBarTok, 128);
+      named_sync(kBarTok, NTOK);
       if (warp == 4 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
         const bool vok = v_zero || wait_bar(x, B_V, (uint32_t)t & 1u);
         if (__shfl_sync(0xffffffffu, vok, 0)) {
@@ -662,7 +681,6 @@ __global__ void __launch_bounds__(NT, 1)
           mma_commit_warp(&x.bar[B_UW]);
         }
       }
-      // W~ from TMEM: thread tt = key channel c writes row c of W~ stored [c][r]
       const bool uw = wait_bar(x, B_UW, (uint32_t)t & 1u);
       tc_fence_after();
       if (warp == 4 && __shfl_sync(0xffffffffu, uw, 0) && t + 1 < nchunks) {  // the U MMA has consumed v
@@ -670,20 +688,21 @@ __global__ void __launch_bounds__(NT, 1)
         if (!v_zero) v_issued = t + 1;
       }
       {
-        // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand block
-        float w[32];
-        tmem_ld32(tl + tW, w);
+        // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand
+        // block: lane quarter = channel block, half = which 16 rows r
+        float w[16];
+        tmem_ld16(tl + tW + 16 * half, w);
         tmem_ld_wait();
-        const int c = tt, h = c >> 6, cc = c & 63;
+        const int c = 32 * quarter + lane, h = c >> 6, cc = c & 63;
         unsigned char *nw = sm + kQKW + pb * 32768 + h * 16384 + 12288;
 #pragma unroll
-        for (int r = 0; r < C; ++r)
-          *reinterpret_cast<__nv_bfloat16 *>(nw + sw128_off(r, cc)) = __float2bfloat16_rn(-w[r]);
+        for (int i = 0; i < 16; ++i)
+          *reinterpret_cast<__nv_bfloat16 *>(nw + sw128_off(16 * half + i, cc)) = __float2bfloat16_rn(-w[i]);
       }
-      if (tt < C) bet[tt] = beta_next;  // the solve of chunk t has read beta(t)
+      if (tt < C) bet[tt] = __bfloat162float(__ushort_as_bfloat16(beta_next));  // beta(t) is no longer read
       fence_proxy_async_smem();
       tc_fence_before();
-      const bool go = named_sync_and(kBarTok, 128, *x.abort == 0);
+      const bool go = named_sync_and(kBarTok, NTOK, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_WT0 + pb]);
       if (!go) break;
     }
@@ -785,8 +804,10 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mg;
   const int BH = a.B * a.H;
   const uint64_t T = (uint64_t)(a.T > 0 ? a.T : 1), n = (uint64_t)BH;
+  CUtensorMap mo;
   if (!encode_tmap_bf16_3d(&mq, a.q, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mk, a.k, D, T, n, 64, C) ||
-      !encode_tmap_bf16_3d(&mv, a.v, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mg, a.g, D, T, n, 64, C))
+      !encode_tmap_bf16_3d(&mv, a.v, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mg, a.g, D, T, n, 64, C) ||
+      !encode_tmap_bf16_3d(&mo, a.o, D, T, n, 64, C))
     return cudaErrorInvalidValue;
   TcParams p;
   p.beta = (const __nv_bfloat16 *)a.beta;
@@ -805,7 +826,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
     p.seg_len = a.T > 0 ? a.T : 1;
     p.nseg = 1;
     p.mode = kModeChain;
-    chunk_tc_kernel<<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+    chunk_tc_kernel<<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();
   }
   const size_t mat = (size_t)D * D;
@@ -820,7 +841,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.st_out = Sw;
   p.sin = Sin;
   p.mode = kModeSegTransition;
-  chunk_tc_kernel<<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+  chunk_tc_kernel<<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int scan_smem = (128 * 129 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
@@ -828,7 +849,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, P);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.mode = kModeSegFinal;
-  chunk_tc_kernel<<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, p);
+  chunk_tc_kernel<<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   return cudaGetLastError();
 }
 
