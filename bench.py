@@ -241,6 +241,10 @@ def main():
     flops = synth.flops_per_token_head(dk, dv, 64) * B * H * T
     tflops = flops / (kern_ms / 1e3) / 1e12
     kernel_name = "chunk16_kernel" if plan["path"] == kda.KDA_PATH_SIMT16 else "chunk_tc_kernel"
+    # With in-device context parallelism one step is three launches (segment
+    # transitions, the prefix scan, the final pass); the roofline then uses the
+    # whole step's time, which is the conservative reading.
+    roofline_scope = "kernel" if plan["launches"] == 1 else "step (%d launches)" % plan["launches"]
     src = (["gated_delta_rule_117_b200/csrc/kda_chunk_simt.cu"] if plan["path"] == kda.KDA_PATH_SIMT16
            else ["gated_delta_rule_117_b200/csrc/kda_chunk_tc.cu"])
     trec = traffic_record("%s:%s" % (kernel_name, w.name), src)
@@ -260,7 +264,8 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single"},
         "tflops": {"value": tflops, "flop_per_token_head": synth.flops_per_token_head(dk, dv, 64),
                    "frac_of_bf16_peak": tflops / pk["bf16_tflops"], "peak_kind": pk_kind},
-        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+        "roofline": {"kernel": kernel_name, "scope": roofline_scope, "bound": "hbm", "achieved": achieved,
+                     "peak": pk["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes_per_launch": bytes_per_launch, "peak_kind": pk_kind,
                      "kernel_ms": kern_ms},

@@ -125,6 +125,26 @@ def head_inputs(w: Workload, b: int, h: int, T: Optional[int] = None) -> Dict[st
                 g=round_to(g, w.dtype), beta=round_to(beta, w.dtype), h0=h0)
 
 
+def head_input_blocks(w: Workload, b: int, h: int, T: Optional[int] = None, block: int = 65536):
+    """The stored inputs of one (b, h) chain in token blocks (same values as
+    head_inputs: every stream is drawn sequentially).  Yields (t0, dict) with
+    q, k, g [n, dk], v [n, dv], beta [n]; h0 is not included."""
+    T = w.T if T is None else T
+    rq, rk, rv, rz, rb = (_rng(w, i, b, h) for i in (_Q, _K, _V, _Z, _BETA))
+    eA = np.exp(decay_log_scale(w, h))[None, :]
+    for t0 in range(0, T, block):
+        n = min(block, T - t0)
+        q = rq.standard_normal((n, w.dk))
+        k = rk.standard_normal((n, w.dk))
+        q /= np.linalg.norm(q, axis=1, keepdims=True)
+        k /= np.linalg.norm(k, axis=1, keepdims=True)
+        v = rv.standard_normal((n, w.dv))
+        g = G_MIN * _sigmoid(eA * rz.standard_normal((n, w.dk)))
+        beta = _sigmoid(rb.standard_normal(n))
+        yield t0, dict(q=round_to(q, w.dtype), k=round_to(k, w.dtype), v=round_to(v, w.dtype),
+                       g=round_to(g, w.dtype), beta=round_to(beta, w.dtype))
+
+
 def _to_torch(x: np.ndarray, dtype) -> torch.Tensor:
     return torch.from_numpy(x).to(dtype)
 
@@ -147,6 +167,39 @@ def prefill_inputs(w: Workload, T: Optional[int] = None, heads=None) -> Dict[str
             for name in ("q", "k", "v", "g", "beta"):
                 out[name][b, h] = _to_torch(x[name], dt)
             out["h0"][b, h] = _to_torch(x["h0"], torch.float32)
+    return out
+
+
+def _fill_heads(args):
+    w, T, heads, tensors = args
+    for b, h in heads:
+        for t0, x in head_input_blocks(w, b, h, T):
+            n = x["beta"].shape[0]
+            for name in ("q", "k", "v", "g", "beta"):
+                tensors[name][b, h, t0:t0 + n] = _to_torch(x[name], w.torch_dtype)
+        if w.h0_std > 0:
+            h0 = round_to(w.h0_std * _rng(w, _H0, b, h).standard_normal((w.dk, w.dv)), "f32")
+            tensors["h0"][b, h] = _to_torch(h0, torch.float32)
+    return len(heads)
+
+
+def prefill_inputs_parallel(w: Workload, workers: int, T: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """prefill_inputs computed by a pool of `workers` spawned processes writing
+    into shared-memory tensors in token blocks (same values, bit for bit)."""
+    assert not w.decode
+    T = w.T if T is None else T
+    dt = w.torch_dtype
+    out = dict(q=torch.empty(w.B, w.H, T, w.dk, dtype=dt), k=torch.empty(w.B, w.H, T, w.dk, dtype=dt),
+               v=torch.empty(w.B, w.H, T, w.dv, dtype=dt), g=torch.empty(w.B, w.H, T, w.dk, dtype=dt),
+               beta=torch.empty(w.B, w.H, T, dtype=dt), h0=torch.zeros(w.B, w.H, w.dk, w.dv, dtype=torch.float32))
+    for t in out.values():
+        t.share_memory_()
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    workers = max(1, min(workers, len(heads)))
+    parts = [heads[i::workers] for i in range(workers)]
+    ctx = torch.multiprocessing.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        pool.map(_fill_heads, [(w, T, part, out) for part in parts])
     return out
 
 

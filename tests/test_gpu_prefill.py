@@ -138,6 +138,20 @@ def test_long_workload_reduced_T():
     assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
 
 
+def test_long_workload_full_sampled_head():
+    # the 1M-token workload at full size (16 chains, the context-parallel plan
+    # the benchmark times); the oracle recomputes one sampled chain end to end
+    import os
+    w = synth.WORKLOADS["long_h16_t1m"]
+    x = synth.prefill_inputs_parallel(w, workers=min(os.cpu_count() or 1, 16))
+    o, hT = _run(x, use_h0=False)
+    assert kda.kda_chunk_fwd_plan(w.B, w.H, w.T, 128, 128, kda.KDA_DTYPE_BF16, 0)["segments"] > 1
+    h = 5
+    o_ref, h_ref = oracle_prefill({k: v[:, h:h + 1] for k, v in x.items()}, h0=False)
+    assert rel_l2(o[:, h:h + 1], o_ref) <= TOL["bf16"] and rel_l2(hT[:, h:h + 1], h_ref) <= TOL["bf16"]
+    assert torch.isfinite(o).all() and torch.isfinite(hT).all()
+
+
 def test_zero_length_copies_state():
     w = synth.WORKLOADS["tiny_f32"].with_(T=0, h0_std=0.02)
     x = synth.prefill_inputs(w)

@@ -88,3 +88,19 @@ def test_algorithmic_counts():
     assert synth.prefill_bytes(w) == 16 * (4096 * 1282 + 2 * 65536)
     d = synth.WORKLOADS["decode_b256_h32"]
     assert synth.decode_bytes_per_step(d) == 256 * 32 * 132354
+
+
+def test_parallel_generation_is_bitwise_identical():
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(H=4, T=96)
+    a = synth.prefill_inputs(w)
+    b = synth.prefill_inputs_parallel(w, workers=3)
+    assert all(torch.equal(a[n], b[n]) for n in a)
+
+
+def test_block_generation_matches_whole_draw():
+    w = synth.WORKLOADS["long_h16_t1m"].with_(T=300)
+    whole = synth.head_inputs(w, 0, 3)
+    parts = list(synth.head_input_blocks(w, 0, 3, block=128))
+    assert [t0 for t0, _ in parts] == [0, 128, 256]
+    for name in ("q", "k", "v", "g", "beta"):
+        assert np.array_equal(np.concatenate([x[name] for _, x in parts]), whole[name])
