@@ -30,20 +30,26 @@
 // tcgen05.mma carries a fixed cost that dominates small-N products.
 //
 // Work split (the report's token-parallel stage vs head-parallel recurrence,
-// section 5.1.1, mapped onto one CTA per (b, h) chain), 8 warps:
-//   warps 0-3  chain:  thread e keeps column e of the fp32 state S in
-//                      registers; per chunk it writes S~^T, issues the V~/O
-//                      MMAs, turns V~^T into bf16 hi/lo operands, issues the
-//                      dS/O MMAs, applies the state update and stores the
-//                      output tile;
-//   warps 4-7  token:  one chunk ahead of the chain: TMA loads, cumulative
-//                      decay and rescaled operands, the Gram MMAs, A, L, the
-//                      triangular solve, the U/W~ MMAs and W~.
-// One elected thread per warpgroup issues its MMAs and TMA copies right after
-// the group's named barrier.  The two groups hand chunks over through
-// mbarriers; buffers the chain reads are double buffered by chunk parity.
-// Every wait is bounded; a wait that gives up sets the device status word and
-// the whole CTA drains without further MMAs.
+// section 5.1.1, mapped onto one CTA per (b, h) chain), 12 warps in three
+// warpgroups that form a pipeline over chunks:
+//   warps 0-3   chain:   thread e keeps column e of the fp32 state S in
+//                        registers (248 registers via setmaxnreg); per chunk
+//                        it writes S~^T, issues the [O | V~] MMAs, turns V~^T
+//                        into bf16 hi/lo operands, issues the dS/O MMAs,
+//                        applies the state update and stores the output tile;
+//   warps 4-7   token A: TMA loads of q, k, g, the cumulative decay, the
+//                        rescaled operands and the Gram MMAs (chunk t + 2);
+//   warps 8-11  token B: A, L, the triangular solve, the U/W~ MMAs and -W~
+//                        (chunk t + 1).
+// One elected lane of a converged warp issues each MMA and TMA copy.  The
+// groups hand chunks over through mbarrier rings indexed by chunk parity;
+// the buffers a later stage reads are double buffered (the per-channel decay
+// factors, which the chain reads last, triple buffered).  The chain hands a
+// chunk's operand buffers back through the commit of the MMAs that read them,
+// and takes the next chunk's e^rho straight from token A, so no stage waits
+// for a later stage of the previous chunk.  Every wait is
+// bounded; a wait that gives up sets the device status word and the whole CTA
+// drains without further MMAs.
 #include <cuda_bf16.h>
 
 #include "kda_internal.cuh"
@@ -58,9 +64,8 @@ using namespace sm100;
 constexpr int C = 32;     // tokens per chunk
 constexpr int D = 128;    // dk = dv
 constexpr int NT = 384;   // 12 warps: chain warpgroup + two token warpgroups
-constexpr int NTOK = 256;  // token-stage threads
 constexpr uint32_t kWaitLimit = 1u << 22;  // polls; seconds, far beyond any real wait
-constexpr uint32_t kBarChain = 1, kBarTok = 2;
+constexpr uint32_t kBarChain = 1, kBarTokA = 2, kBarTokB = 3;
 
 // ---- shared memory (byte offsets from a 1024-aligned base) -------------------
 // "h0/h1" = channel blocks 0..63 / 64..127 of a [tokens x 128] bf16 tile stored
@@ -79,33 +84,46 @@ constexpr int kLf = 190464;      // fp32 L [32][33]
 constexpr int kNf = 194688;      // fp32 N = (I + L)^-1 [32][33]
 constexpr int kXf = 198912;      // fp32 scratch [16][17]
 constexpr int kXa = 200000;      // fp32 [32][33]: Qs_lo Kc_hi part of A
-constexpr int kFac = 204224;     // [2]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
-constexpr int kXch = 207296;     // fp32 [4][128]: per-quarter sums of g (8 tokens each)
-constexpr int kBeta = 209344;    // fp32 beta[32]
-constexpr int kBar = 209472;     // mbarriers
-constexpr int kMisc = 209728;    // TMEM base address, abort flag
-constexpr int kOst = 210944;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
-constexpr int kSmemBytes = 219136 + 1024;
+constexpr int kFac = 204224;     // [3]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
+constexpr int kXch = 208832;     // fp32 [2][128]: per-half sums of g (16 tokens each)
+constexpr int kBeta = 209856;    // [2]: fp32 beta[32] (written by token A, read by token B)
+constexpr int kBar = 210112;     // mbarriers
+constexpr int kMisc = 210240;    // TMEM base address, abort flag
+constexpr int kOst = 211968;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
+constexpr int kSmemBytes = 220160 + 1024;
+// each region ends where the next begins (or before)
+static_assert(kRawQK + 16384 <= kRawG && kRawG + 8192 <= kRawV && kRawV + 8192 <= kQKW, "smem layout");
+static_assert(kQKW + 2 * 32768 <= kKC && kKC + 2 * 16384 <= kST && kST + 32768 <= kVTH, "smem layout");
+static_assert(kVTH + 8192 <= kVTL && kVTL + 8192 <= kAH && kAH + 2 * 4096 <= kTT && kTT + 2048 <= kLf, "smem layout");
+static_assert(kLf + 4224 <= kNf && kNf + 4224 <= kXf && kXf + 16 * 17 * 4 <= kXa && kXa + 4224 <= kFac, "smem layout");
+static_assert(kFac + 3 * 1536 <= kXch && kXch + 2 * 128 * 4 <= kBeta && kBeta + 2 * 128 <= kBar, "smem layout");
+static_assert(kBar + 8 * 16 <= kMisc && kMisc + 8 <= kOst && kOst + 8192 + 1024 <= kSmemBytes, "smem layout");
+static_assert(kOst % 1024 == 0 && kQKW % 1024 == 0 && kKC % 1024 == 0 && kST % 1024 == 0, "swizzled tiles");
+static_assert(kSmemBytes <= 232448, "over the per-CTA shared memory limit");
 
-// barrier slots
+// barrier slots ([2] = ring indexed by chunk parity)
 enum {
   B_QKG = 0,   // q,k,g of the chunk landed (TMA)
   B_V,         // v of the chunk landed (TMA)
-  B_GRAM,      // Gram MMAs done
+  B_DEC0,      // [2] token A: operands, factors and beta of the chunk written
+  B_DEC1,
+  B_GRAM0,     // [2] Gram MMAs of the chunk done
+  B_GRAM1,
   B_UW,        // U, W~ MMAs done
-  B_WT0,       // [2] token: chunk ready for the chain (W~, U, operands, factors)
+  B_WT0,       // [2] token B: chunk ready for the chain (W~, U, A)
   B_WT1,
-  B_V1,        // V~ and O-inter MMAs done
+  B_V1,        // [O | V~] MMAs done
   B_DS,        // dS and O-intra MMAs done
-  B_CD0,       // [2] chain finished with the chunk's buffers
+  B_CD0,       // [2] the chain's MMAs have read the chunk's operands (tcgen05.commit)
   B_CD1,
   B_COUNT
 };
+static_assert(B_COUNT <= 16, "mbarrier region holds 16 barriers");
 
 // TMEM columns (fp32, 128 lanes).  The output and pseudo-value accumulators
 // of a chunk parity are adjacent ([O | U]) so one N = 64 MMA updates both.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t tG = 0, tOU = 64, tW = 192, tDS = 256;  // tO(p) = tOU + 64 p, tU(p) = tO(p) + 32
+constexpr uint32_t tG0 = 0, tG1 = 384, tOU = 64, tW = 192, tDS = 256;  // tO(p) = tOU + 64 p, tU(p) = tO(p) + 32
 
 // Launch modes.  kModeChain: one CTA per (b, h) chain over all T tokens.
 // In-device context parallelism (the report's section 5.1.1 SM-level CP,
@@ -166,55 +184,42 @@ __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// ---- token stage: one chunk, 256 threads (tt = 0..255) ------------------------
-// Thread tt owns the key-channel pair (2pp, 2pp+1) for the 8 tokens of
-// quarter qt of the chunk.  The chunk-local cumulative decay is assembled from
-// the quarters' sums (exchanged through shared memory).  All shared-memory
-// reads are staged into registers before the first store so they are not
-// serialised behind possibly-aliasing stores.
-__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
+// ---- token A: decay and rescaled operands of one chunk, 128 threads ----------
+// Thread tt owns the key-channel pair (2pp, 2pp+1) for the 16 tokens of half
+// hf of the chunk.  The token loops are kept rolled: three warpgroups share
+// each SM sub-partition's instruction cache, so code size costs time here.
+__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs) {
   unsigned char *sm = x.sm;
-  const int pp = tt & 63, qt = tt >> 6;
+  const int pp = tt & 63, hf = tt >> 6;
   const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
-  uint32_t graw[8], qraw[8], kraw[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t off = h * 4096 + sw128_off(8 * qt + i, cc);
-    graw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawG + off);
-    qraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + off);
-    kraw[i] = *reinterpret_cast<const uint32_t *>(sm + kRawQK + 8192 + off);
+  const unsigned char *rg = sm + kRawG + h * 4096;
+  const unsigned char *rq = sm + kRawQK + h * 4096;
+  const unsigned char *rk = sm + kRawQK + 8192 + h * 4096;
+  // sum of g over the half
+  float S0 = 0.f, S1 = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rg + sw128_off(16 * hf + i, cc)));
+    S0 += g.x;
+    S1 += g.y;
   }
-  float xs0[8], xs1[8];
-  float G0 = 0.f, G1 = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&graw[i]));
-    G0 += g.x;
-    G1 += g.y;
-    xs0[i] = G0;
-    xs1[i] = G1;
-  }
-  float *xq = reinterpret_cast<float *>(sm + kXch);  // [quarter][channel] sums
-  *reinterpret_cast<float2 *>(xq + 128 * qt + c0) = make_float2(G0, G1);
-  named_sync(kBarTok, NTOK);
-  // x = G_s - G_15 with G_15 = (sum of quarters 0, 1): quarter offsets
-  float o0, o1;
-  {
-    const float2 s0 = *reinterpret_cast<const float2 *>(xq + c0);
-    const float2 s1 = *reinterpret_cast<const float2 *>(xq + 128 + c0);
-    const float2 s2 = *reinterpret_cast<const float2 *>(xq + 256 + c0);
-    o0 = qt == 0 ? -(s0.x + s1.x) : qt == 1 ? -s1.x : qt == 2 ? 0.f : s2.x;
-    o1 = qt == 0 ? -(s0.y + s1.y) : qt == 1 ? -s1.y : qt == 2 ? 0.f : s2.y;
-  }
+  float *xch = reinterpret_cast<float *>(sm + kXch);
+  *reinterpret_cast<float2 *>(xch + 128 * hf + c0) = make_float2(S0, S1);
+  // tokens 0..15: x = G_s - G_15 (>= 0); tokens 16..31: x = sum_{16..s} g (<= 0)
+  const float b0 = hf == 0 ? S0 : 0.f, b1 = hf == 0 ? S1 : 0.f;
   unsigned char *qkw = sm + kQKW + p * 32768 + h * 16384;  // Ks | Qs lo | Qs | -W~
   unsigned char *kc = sm + kKC + p * 16384 + h * 8192;     // Kc hi | Kc lo
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t off = sw128_off(8 * qt + i, cc);
-    const float x0 = fminf(fmaxf(xs0[i] + o0, -87.f), 87.f), x1 = fminf(fmaxf(xs1[i] + o1, -87.f), 87.f);
+  float P0 = 0.f, P1 = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t off = sw128_off(16 * hf + i, cc);
+    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rg + off));
+    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rq + off));
+    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rk + off));
+    P0 += g.x;
+    P1 += g.y;
+    const float x0 = fminf(fmaxf(P0 - b0, -87.f), 87.f), x1 = fminf(fmaxf(P1 - b1, -87.f), 87.f);
     const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
-    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qraw[i]));
-    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kraw[i]));
     uint32_t qlo, clo;
     const uint32_t qhi = split2(q.x * e0, q.y * e1, qlo);
     const __nv_bfloat162 khi = __floats2bfloat162_rn(k.x * e0, k.y * e1);
@@ -225,10 +230,11 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
     *reinterpret_cast<uint32_t *>(kc + off) = chi;
     *reinterpret_cast<uint32_t *>(kc + 4096 + off) = clo;
   }
-  if (tt < 128) {
+  named_sync(kBarTokA, 128);
+  {
     const int c = tt;
-    float *fac = reinterpret_cast<float *>(sm + kFac + p * 1536);
-    const float rho = xq[c] + xq[128 + c], tail = xq[256 + c] + xq[384 + c];
+    float *fac = reinterpret_cast<float *>(sm + kFac + fs * 1536);
+    const float rho = xch[c], tail = xch[128 + c];
     fac[c] = __expf(rho);                // e^rho
     fac[128 + c] = __expf(rho + tail);   // e^{G_31}
     fac[256 + c] = __expf(tail);         // e^{G_31 - rho}
@@ -236,13 +242,12 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p) {
 }
 
 // N = (I + L)^-1 for the strictly lower 32x32 L in Lf (fp32), blocked 8 -> 16 -> 32,
-// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  256 threads.
-__device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
+// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  Token B, 128 threads.
+__device__ __forceinline__ void token_solve(const Ctx &x, int tt, const float *bet) {
   unsigned char *sm = x.sm;
   const float *L = reinterpret_cast<const float *>(sm + kLf);
   float *N = reinterpret_cast<float *>(sm + kNf);
   float *X = reinterpret_cast<float *>(sm + kXf);
-  const float *bet = reinterpret_cast<const float *>(sm + kBeta);
   // level 1: the four 8x8 diagonal blocks, one column per thread
   if (tt < 32) {
     const int q = tt >> 3, jj = tt & 7, b0 = 8 * q;
@@ -256,54 +261,56 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt) {
       N[(b0 + r) * 33 + b0 + jj] = acc;
     }
   }
-  named_sync(kBarTok, NTOK);
+  named_sync(kBarTokB, 128);
   // level 2: N_10 = -N_11 L_10 N_00 inside each 16x16 block (8x8 pieces)
-  if (tt < 128) {
+  {
     const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) acc += L[(o + 8 + r) * 33 + o + s] * N[(o + s) * 33 + o + j];
     X[blk * 64 + e] = acc;
   }
-  named_sync(kBarTok, NTOK);
-  if (tt < 128) {
+  named_sync(kBarTokB, 128);
+  {
     const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 8; ++s) acc += N[(o + 8 + r) * 33 + o + 8 + s] * X[blk * 64 + s * 8 + j];
     N[(o + 8 + r) * 33 + o + j] = -acc;
   }
-  named_sync(kBarTok, NTOK);
-  // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (one element per thread)
-  {
-    const int r = tt >> 4, j = tt & 15;
+  named_sync(kBarTokB, 128);
+  // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (2 elements per thread)
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += L[(16 + r) * 33 + s] * N[s * 33 + j];
     X[r * 17 + j] = acc;
   }
-  named_sync(kBarTok, NTOK);
-  {
-    const int r = tt >> 4, j = tt & 15;
+  named_sync(kBarTokB, 128);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
     float acc = 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) acc += N[(16 + r) * 33 + 16 + s] * X[s * 17 + j];
     N[(16 + r) * 33 + j] = -acc;
   }
-  named_sync(kBarTok, NTOK);
-  // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 4-column piece)
+  named_sync(kBarTokB, 128);
+  // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 8-column chunk k)
   {
-    const int r = tt >> 3, k = (tt >> 1) & 3, half = tt & 1;
-    uint2 w;
+    const int r = tt >> 2, k = tt & 3;
+    uint4 w;
     uint32_t *pw = &w.x;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int j0 = 8 * k + 4 * half + 2 * i;
+    for (int i = 0; i < 4; ++i) {
+      const int j0 = 8 * k + 2 * i;
       const float a0 = (j0 <= r) ? N[r * 33 + j0] * bet[j0] : 0.f;
       const float a1 = (j0 + 1 <= r) ? N[r * 33 + j0 + 1] * bet[j0 + 1] : 0.f;
       pw[i] = pack_bf16x2(a0, a1);
     }
-    *reinterpret_cast<uint2 *>(sm + kTT + sw64_chunk(r, k) + 8 * half) = w;
+    *reinterpret_cast<uint4 *>(sm + kTT + sw64_chunk(r, k)) = w;
   }
 }
 
@@ -469,14 +476,15 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
         mma_commit_warp(&x.bar[B_DS]);
+        // once these MMAs have read them, chunk t's operand buffers may take chunk t + 2
+        mma_commit_warp(&x.bar[B_CD0 + pb]);
       }
-      // the next chunk's factors are needed to write S~^T(t+1) in the update pass
-      bool next_ready = true;
-      if (has_next) next_ready = wait_bar(x, B_WT0 + (pb ^ 1), (uint32_t)((t + 1) >> 1) & 1u);
+      // the next chunk's e^rho (written by token A) is needed to form S~^T(t+1)
+      if (has_next) wait_bar(x, B_DEC0 + (pb ^ 1), (uint32_t)((t + 1) >> 1) & 1u);
       wait_bar(x, B_DS, (uint32_t)t & 1u);
       tc_fence_after();
       {
-        const float *fac = reinterpret_cast<const float *>(sm + kFac + pb * 1536);
+        const float *fac = reinterpret_cast<const float *>(sm + kFac + (t % 3) * 1536);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float ds[32];
@@ -495,15 +503,21 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       if (has_next) {
-        const float *erho = reinterpret_cast<const float *>(sm + kFac + (pb ^ 1) * 1536);
+        const float *erho = reinterpret_cast<const float *>(sm + kFac + ((t + 1) % 3) * 1536);
 #pragma unroll
         for (int q = 0; q < 4; ++q) store_st32(st, erho, S, e, q);
         fence_proxy_async_smem();
       }
       tc_fence_before();
       const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
-      if (e == 0) mbar_arrive(&x.bar[B_CD0 + pb]);  // chunk t's buffers are free for chunk t + 2
-      if (warp == 0 && __shfl_sync(0xffffffffu, has_next && next_ready && go, 0)) issue_v1(t + 1);
+      // [O | V~](t+1) is issued as soon as token B has finished chunk t + 1;
+      // if it has not yet, the output tile of chunk t goes out first
+      const uint32_t wt_next = B_WT0 + (pb ^ 1), wt_par = (uint32_t)((t + 1) >> 1) & 1u;
+      bool issued = !(has_next && go);
+      if (warp == 0 && !issued && __shfl_sync(0xffffffffu, mbar_try_wait(&x.bar[wt_next], wt_par), 0)) {
+        issue_v1(t + 1);
+        issued = true;
+      }
       // output tile of chunk t (its TMEM half is not touched by chunk t + 1):
       // column e goes into a swizzled shared tile that one TMA store writes out
       // (rows past the end of the sequence are clipped by the tensor map)
@@ -524,6 +538,7 @@ __global__ void __launch_bounds__(NT, 1)
           if (lane == 0) bulk_wait_read_all();  // the tile is rewritten next chunk
         }
       }
+      if (warp == 0 && !issued && __shfl_sync(0xffffffffu, wait_bar(x, wt_next, wt_par), 0)) issue_v1(t + 1);
       tc_fence_before();
       if (!go) break;
     }
@@ -532,15 +547,13 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int c = 0; c < D; ++c) hdst[c * D + e] = S[c];
     }
-  } else {
-    // ======================= token warpgroups (8 warps) =======================
+  } else if (warp < 8) {
+    // ======================= token A (warps 4-7) =======================
     regs_decrease<120>();
     const int tt = tid - 128;
-    const int quarter = warp & 3, half = (warp >> 3) & 1;  // TMEM lane quarter; which half of the columns
-    const uint32_t tl = tbase + ((uint32_t)(32 * quarter) << 16);
     const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
+    const unsigned short *beta_bits = reinterpret_cast<const unsigned short *>(beta);
     const uint32_t idG = idesc_bf16(128, 64, false, false, false);
-    const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
     // TMA issue, called by all of warp 4 (one elected lane issues).
     auto tma_qkg = [&](int t) {
       mbar_arrive_expect_tx_warp(&x.bar[B_QKG], 6 * 4096);
@@ -552,6 +565,60 @@ __global__ void __launch_bounds__(NT, 1)
       tma_load_3d_warp(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
       tma_load_3d_warp(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
     };
+    int qkg_issued = -1;  // last chunk whose q, k, g copy was issued (abort path)
+    if (warp == 4 && nchunks > 0) {
+      if (lane == 0) {
+        prefetch_tmap(&mq);
+        prefetch_tmap(&mk);
+        prefetch_tmap(&mg);
+      }
+      tma_qkg(0);
+      qkg_issued = 0;
+    }
+    // beta(t) is loaded from global one chunk ahead and handed to token B in
+    // shared memory (double buffered by chunk parity)
+    unsigned short beta_cur = 0;
+    if (tt < C && tb + tt < te) beta_cur = __ldg(beta_bits + tb + tt);
+    for (int t = 0; t < nchunks; ++t) {
+      const int pb = t & 1, t0 = tb + t * C;
+      unsigned short beta_next = 0;
+      if (tt < C && t0 + C + tt < te) beta_next = __ldg(beta_bits + t0 + C + tt);
+      if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);  // chunk t-2's buffers are free
+      const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
+      if (tt < C) reinterpret_cast<float *>(sm + kBeta + pb * 128)[tt] = __bfloat162float(__ushort_as_bfloat16(beta_cur));
+      token_decay(x, tt, pb, t % 3);
+      fence_proxy_async_smem();
+      const bool go = named_sync_and(kBarTokA, 128, *x.abort == 0);
+      if (tt == 0) mbar_arrive(&x.bar[B_DEC0 + pb]);
+      if (warp == 4 && __shfl_sync(0xffffffffu, landed && go, 0)) {
+        tc_fence_after();
+        // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
+        const uint64_t dA = sdesc_sw128(sbase + kQKW + pb * 32768, 16, 1024);
+        const uint64_t dB = sdesc_sw128(sbase + kKC + pb * 16384, 16, 1024);
+        const uint32_t tg = tbase + (pb ? tG1 : tG0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_warp(tg, sdesc_add(dA, (ks >> 2) * 16384 + (ks & 3) * 32),
+                        sdesc_add(dB, (ks >> 2) * 8192 + (ks & 3) * 32), idG, ks > 0);
+        mma_commit_warp(&x.bar[B_GRAM0 + pb]);
+        if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
+          tma_qkg(t + 1);
+          qkg_issued = t + 1;
+        }
+      }
+      beta_cur = beta_next;
+      if (!go) break;
+    }
+    if (tt == 0 && *x.abort && qkg_issued >= 0)  // let the last q, k, g copy land before the CTA exits
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_QKG], (uint32_t)qkg_issued & 1u); ++i) {
+      }
+  } else {
+    // ======================= token B (warps 8-11) =======================
+    regs_decrease<120>();
+    const int tt = tid - 256;
+    const int quarter = warp & 3;  // TMEM lane quarter
+    const uint32_t tl = tbase + ((uint32_t)(32 * quarter) << 16);
+    const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
     auto tma_v = [&](int t) {
       if (v_zero) return;  // transition runs: v = 0, the buffer holds zeros
       mbar_arrive_expect_tx_warp(&x.bar[B_V], 2 * 4096);
@@ -562,97 +629,63 @@ __global__ void __launch_bounds__(NT, 1)
     // 16x16 products read them: they must hold zeros.
     {
       float *N = reinterpret_cast<float *>(sm + kNf);
-      for (int i = tt; i < 32 * 33; i += NTOK) N[i] = 0.f;
+      for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
       if (v_zero) {  // v = 0 for a transition run: the U MMA then yields U = 0
         uint4 *zv = reinterpret_cast<uint4 *>(sm + kRawV);
-        for (int i = tt; i < 512; i += NTOK) zv[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tt; i < 512; i += 128) zv[i] = make_uint4(0, 0, 0, 0);
       }
-      named_sync(kBarTok, NTOK);
+      named_sync(kBarTokB, 128);
     }
-    // TMA copies issued and not yet waited for (the abort path lets them land).
-    int qkg_issued = -1, v_issued = -1;
-    if (warp == 4 && nchunks > 0) {
-      if (lane == 0) {
-        prefetch_tmap(&mq);
-        prefetch_tmap(&mk);
-        prefetch_tmap(&mv);
-        prefetch_tmap(&mg);
-      }
-      tma_qkg(0);
+    int v_issued = -1;  // last chunk whose v copy was issued (abort path)
+    if (warp == 8 && nchunks > 0) {
+      if (lane == 0) prefetch_tmap(&mv);
       tma_v(0);
-      qkg_issued = 0;
       v_issued = v_zero ? -1 : 0;
     }
-    // beta goes through shared memory one chunk ahead: the global load for
-    // chunk t + 1 is issued at the top of chunk t and converted at its end.
-    float *bet = reinterpret_cast<float *>(sm + kBeta);
-    const unsigned short *beta_bits = reinterpret_cast<const unsigned short *>(beta);
-    if (tt < C) bet[tt] = (tb + tt < te) ? __bfloat162float(beta[tb + tt]) : 0.f;
     for (int t = 0; t < nchunks; ++t) {
-      const int pb = t & 1, t0 = tb + t * C;
-      unsigned short beta_next = 0;
-      if (tt < C && t0 + C + tt < te) beta_next = __ldg(beta_bits + t0 + C + tt);
-      if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);
-      const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
-      token_decay(x, tt, pb);
-      fence_proxy_async_smem();
-      named_sync(kBarTok, NTOK);
-      if (warp == 4 && __shfl_sync(0xffffffffu, landed && !*x.abort, 0)) {
-        tc_fence_after();
-        // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
-        const uint64_t dA = sdesc_sw128(sbase + kQKW + pb * 32768, 16, 1024);
-        const uint64_t dB = sdesc_sw128(sbase + kKC + pb * 16384, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_bf16_warp(tbase + tG, sdesc_add(dA, (ks >> 2) * 16384 + (ks & 3) * 32),
-                        sdesc_add(dB, (ks >> 2) * 8192 + (ks & 3) * 32), idG, ks > 0);
-        mma_commit_warp(&x.bar[B_GRAM]);
-        if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
-          tma_qkg(t + 1);
-          qkg_issued = t + 1;
-        }
-      }
-      // Gram tile -> L (lanes 0-31: Ks rows) and A (lanes 64-95: Qs rows, plus
-      // the Qs-lo part from lanes 32-63); two warps per lane quarter, each
-      // taking 16 of the 32 columns j.
-      wait_bar(x, B_GRAM, (uint32_t)t & 1u);
+      const int pb = t & 1;
+      const float *bet = reinterpret_cast<const float *>(sm + kBeta + pb * 128);
+      wait_bar(x, B_DEC0 + pb, (uint32_t)(t >> 1) & 1u);
+      wait_bar(x, B_GRAM0 + pb, (uint32_t)(t >> 1) & 1u);
       tc_fence_after();
-      float a[16];
-      const int r = lane, j0 = 16 * half;
+      // Gram tile -> L (lanes 0-31: Ks rows) and A (lanes 64-95: Qs rows, plus
+      // the Qs-lo part from lanes 32-63)
+      const uint32_t tg = (pb ? tG1 : tG0);
+      float a[32];
+      const int r = lane;
       if (quarter == 0 || quarter == 2) {
-        float b[16];
-        tmem_ld16(tl + tG + j0, a);
-        tmem_ld16(tl + tG + 32 + j0, b);
+        float b[32];
+        tmem_ld32(tl + tg, a);
+        tmem_ld32(tl + tg + 32, b);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) a[j] += b[j];
+        for (int j = 0; j < 32; ++j) a[j] += b[j];
         if (quarter == 0) {
           const float br = bet[r];
           float *Lm = reinterpret_cast<float *>(sm + kLf);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) Lm[r * 33 + j0 + j] = (j0 + j < r) ? br * a[j] : 0.f;
+          for (int j = 0; j < 32; ++j) Lm[r * 33 + j] = (j < r) ? br * a[j] : 0.f;
         }
       } else if (quarter == 1) {
-        tmem_ld16(tl + tG + j0, a);
+        tmem_ld32(tl + tg, a);
         tmem_ld_wait();
         float *Xa = reinterpret_cast<float *>(sm + kXa);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) Xa[r * 33 + j0 + j] = a[j];
+        for (int j = 0; j < 32; ++j) Xa[r * 33 + j] = a[j];
       }
       tc_fence_before();
-      named_sync(kBarTok, NTOK);
+      named_sync(kBarTokB, 128);
       if (quarter == 2) {
         const float *Xa = reinterpret_cast<const float *>(sm + kXa);
         unsigned char *ah = sm + kAH + pb * 4096;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int k = 2 * half + kk;
+        for (int k = 0; k < 4; ++k) {
           uint4 hi, lo;
           float m[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int j = 8 * k + i;
-            m[i] = (j <= r) ? a[8 * kk + i] + Xa[r * 33 + j] : 0.f;
+            m[i] = (j <= r) ? a[j] + Xa[r * 33 + j] : 0.f;
           }
           hi.x = split2(m[0], m[1], lo.x);
           hi.y = split2(m[2], m[3], lo.y);
@@ -662,10 +695,10 @@ __global__ void __launch_bounds__(NT, 1)
           *reinterpret_cast<uint4 *>(ah + 2048 + sw64_chunk(r, k)) = lo;
         }
       }
-      token_solve(x, tt);
+      token_solve(x, tt, bet);
       fence_proxy_async_smem();
-      named_sync(kBarTok, NTOK);
-      if (warp == 4 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
+      named_sync(kBarTokB, 128);
+      if (warp == 8 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
         const bool vok = v_zero || wait_bar(x, B_V, (uint32_t)t & 1u);
         if (__shfl_sync(0xffffffffu, vok, 0)) {
           tc_fence_after();
@@ -683,43 +716,42 @@ __global__ void __launch_bounds__(NT, 1)
       }
       const bool uw = wait_bar(x, B_UW, (uint32_t)t & 1u);
       tc_fence_after();
-      if (warp == 4 && __shfl_sync(0xffffffffu, uw, 0) && t + 1 < nchunks) {  // the U MMA has consumed v
+      if (warp == 8 && __shfl_sync(0xffffffffu, uw, 0) && t + 1 < nchunks) {  // the U MMA has consumed v
         tma_v(t + 1);
         if (!v_zero) v_issued = t + 1;
       }
       {
-        // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand
-        // block: lane quarter = channel block, half = which 16 rows r
-        float w[16];
-        tmem_ld16(tl + tW + 16 * half, w);
+        // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand block
+        float w[32];
+        tmem_ld32(tl + tW, w);
         tmem_ld_wait();
-        const int c = 32 * quarter + lane, h = c >> 6, cc = c & 63;
+        const int c = tt, h = c >> 6, cc = c & 63;
         unsigned char *nw = sm + kQKW + pb * 32768 + h * 16384 + 12288;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          *reinterpret_cast<__nv_bfloat16 *>(nw + sw128_off(16 * half + i, cc)) = __float2bfloat16_rn(-w[i]);
+        for (int i = 0; i < C; ++i)
+          *reinterpret_cast<__nv_bfloat16 *>(nw + sw128_off(i, cc)) = __float2bfloat16_rn(-w[i]);
       }
-      if (tt < C) bet[tt] = __bfloat162float(__ushort_as_bfloat16(beta_next));  // beta(t) is no longer read
       fence_proxy_async_smem();
       tc_fence_before();
-      const bool go = named_sync_and(kBarTok, NTOK, *x.abort == 0);
+      const bool go = named_sync_and(kBarTokB, 128, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_WT0 + pb]);
       if (!go) break;
     }
-    if (tt == 0 && *x.abort) {  // let every TMA already issued land before the CTA exits (warp 4 issued them)
-      if (qkg_issued >= 0)
-        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_QKG], (uint32_t)qkg_issued & 1u); ++i) {
-        }
-      if (v_issued >= 0)
-        for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_V], (uint32_t)v_issued & 1u); ++i) {
-        }
-    }
+    if (tt == 0 && *x.abort && v_issued >= 0)  // let the last v copy land before the CTA exits
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_V], (uint32_t)v_issued & 1u); ++i) {
+      }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 4) {
+    // after an abort an MMA issued before it may still be running: give it
+    // time to retire before its TMEM is released
+    if (*x.abort) {
+      const uint64_t t_start = global_ns();
+      while (global_ns() - t_start < 200000ull) __nanosleep(10000);
+    }
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);
   }
