@@ -89,6 +89,26 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
+    def count(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for line in f if line.count(",") >= 8)
+        except OSError:
+            return 0
+
+    def soak(self, fn, torch, min_samples=3, max_s=4.0):
+        """Run `fn` (the step, untimed) until nvidia-smi has logged a few
+        samples: a timed region of a few milliseconds is far shorter than its
+        sampling period, so the clock record spans this soak of the same work
+        running right before the timed region, plus the timed region itself."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while self.count() < min_samples and time.time() - t0 < max_s:
+            for _ in range(10):
+                fn()
+            torch.cuda.synchronize()
+
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return None
@@ -109,7 +129,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": "soak of the same step just before the timed region, then the timed region"}
 
 
 def rank_workload(w, rank):
@@ -222,6 +242,10 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(gpu_uuid(torch, dev)) as clk:
+        clk.soak(lambda: (flush.zero_(), step()), torch)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         for i in range(args.steps):
             flush.zero_()  # L2 flush between timed iterations (outside the events)
             ev[i][0].record(stream)

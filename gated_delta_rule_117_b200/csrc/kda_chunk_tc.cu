@@ -15,7 +15,9 @@
 //     T  = (I + L)^-1 Diag(beta)               (fp32 blocked substitution)
 //     U  = T V,  W~ = T Ks,  V~ = U - W~ S~     (pseudo-values)
 //     O  = scale (Qs S~ + A V~)
-//     S' = Diag(e^{G_31}) S + Diag(e^{G_31 - rho}) Kc^T V~
+//     S' = Diag(e^{G_31}) S + Diag(e^{G_31 - rho}) Kc^T V~ = Diag(e^{G_31 - rho}) (S~ + Kc^T V~)
+// The chain keeps S~ alone: the next chunk's S~ is Diag(e^{rho'}) Diag(e^{G_31 - rho})
+// (S~ + Kc^T V~), rho' the next chunk's reference (0 after the last chunk).
 // Every tensor-core product is issued "transposed" so that M = 128 is a
 // channel dimension and the TMEM lane is the channel an epilogue thread owns:
 //     Gram  D[.][j|32+j] = [Ks; Qs_lo; Qs; -] [Kc_hi | Kc_lo]^T   (one N = 64 product;
@@ -74,31 +76,35 @@ constexpr int kRawQK = 0;        // q h0 | q h1 | k h0 | k h1 (TMA)
 constexpr int kRawG = 16384;     // g h0 | g h1 (TMA)
 constexpr int kRawV = 24576;     // v h0 | v h1 (TMA; the U MMA reads it in place)
 constexpr int kQKW = 32768;      // [2] x 32 KB; per channel block (16 KB): Ks | Qs lo | Qs | -W~, 4 KB each
-constexpr int kKC = 98304;       // [2] x 16 KB; per channel block (8 KB): Kc hi | Kc lo
-constexpr int kST = 131072;      // S~^T [e][c], K-halves of 16 KB (SW128)
-constexpr int kVTH = 163840;     // V~^T hi [e][j] (SW64, 64-byte rows)
-constexpr int kVTL = 172032;     // V~^T lo
-constexpr int kAH = 180224;      // [2] x 4 KB: A hi [r][j] (SW64) | A lo
-constexpr int kTT = 188416;      // T [r][s] (SW64)
-constexpr int kLf = 190464;      // fp32 L [32][33]
-constexpr int kNf = 194688;      // fp32 N = (I + L)^-1 [32][33]
-constexpr int kXf = 198912;      // fp32 scratch [16][17]
-constexpr int kXa = 200000;      // fp32 [32][33]: Qs_lo Kc_hi part of A
-constexpr int kFac = 204224;     // [3]: fp32 e^rho[128], e^{G_31}[128], e^{G_31-rho}[128] (1536 B each)
-constexpr int kXch = 208832;     // fp32 [2][128]: per-half sums of g (16 tokens each)
-constexpr int kBeta = 209856;    // [2]: fp32 beta[32] (written by token A, read by token B)
-constexpr int kBar = 210112;     // mbarriers
-constexpr int kMisc = 210240;    // TMEM base address, abort flag
-constexpr int kOst = 211968;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
-constexpr int kSmemBytes = 220160 + 1024;
+constexpr int kKC = 98304;       // [3] x 16 KB; per channel block (8 KB): Kc hi | Kc lo
+constexpr int kST = 147456;      // S~^T [e][c], K-halves of 16 KB (SW128)
+// V~^T hi / lo [e][j] (SW64, 64-byte rows) share the S~^T buffer: they are
+// written once the [O | V~] MMAs have consumed S~^T and read by the dS MMAs,
+// which complete before the update writes the next S~^T
+constexpr int kVTH = kST;
+constexpr int kVTL = kST + 8192;
+constexpr int kAH = 180224;      // [3] x 4 KB: A hi [r][j] (SW64) | A lo
+constexpr int kTT = 192512;      // T [r][s] (SW64)
+constexpr int kLf = 194560;      // fp32 L [32][33]
+constexpr int kNf = 198784;      // fp32 N = (I + L)^-1 [32][33]
+constexpr int kXf = 203008;      // fp32 scratch [16][17]
+constexpr int kXa = 204096;      // fp32 [32][33]: Qs_lo Kc_hi part of A
+constexpr int kFac = 208320;     // [3]: fp32 e^rho[128], e^{G_31-rho}[128] (1 KB each)
+constexpr int kXch = 212928;     // fp32 [2][128]: per-half sums of g (16 tokens each)
+constexpr int kBeta = 213952;    // [2]: fp32 beta[32] (written by token A, read by token B)
+constexpr int kBar = 214208;     // mbarriers
+constexpr int kMisc = 214336;    // TMEM base address, abort flag
+constexpr int kOst = 215040;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
+constexpr int kSmemBytes = 223232 + 1024;
 // each region ends where the next begins (or before)
 static_assert(kRawQK + 16384 <= kRawG && kRawG + 8192 <= kRawV && kRawV + 8192 <= kQKW, "smem layout");
-static_assert(kQKW + 2 * 32768 <= kKC && kKC + 2 * 16384 <= kST && kST + 32768 <= kVTH, "smem layout");
-static_assert(kVTH + 8192 <= kVTL && kVTL + 8192 <= kAH && kAH + 2 * 4096 <= kTT && kTT + 2048 <= kLf, "smem layout");
+static_assert(kQKW + 2 * 32768 <= kKC && kKC + 3 * 16384 <= kST && kST + 32768 <= kAH, "smem layout");
+static_assert(kVTL + 8192 <= kST + 32768 && kAH + 3 * 4096 <= kTT && kTT + 2048 <= kLf, "smem layout");
 static_assert(kLf + 4224 <= kNf && kNf + 4224 <= kXf && kXf + 16 * 17 * 4 <= kXa && kXa + 4224 <= kFac, "smem layout");
-static_assert(kFac + 3 * 1536 <= kXch && kXch + 2 * 128 * 4 <= kBeta && kBeta + 2 * 128 <= kBar, "smem layout");
+static_assert(kFac + 3 * 1024 <= kXch && kXch + 2 * 128 * 4 <= kBeta && kBeta + 2 * 128 <= kBar, "smem layout");
 static_assert(kBar + 8 * 16 <= kMisc && kMisc + 8 <= kOst && kOst + 8192 + 1024 <= kSmemBytes, "smem layout");
 static_assert(kOst % 1024 == 0 && kQKW % 1024 == 0 && kKC % 1024 == 0 && kST % 1024 == 0, "swizzled tiles");
+static_assert(kAH % 512 == 0 && kTT % 512 == 0, "64-byte swizzled tiles");
 static_assert(kSmemBytes <= 232448, "over the per-CTA shared memory limit");
 
 // barrier slots ([2] = ring indexed by chunk parity)
@@ -114,7 +120,7 @@ enum {
   B_WT1,
   B_V1,        // [O | V~] MMAs done
   B_DS,        // dS and O-intra MMAs done
-  B_CD0,       // [2] the chain's MMAs have read the chunk's operands (tcgen05.commit)
+  B_CD0,       // [2] the chain's [O | V~] MMAs of the chunk are done (tcgen05.commit)
   B_CD1,
   B_COUNT
 };
@@ -123,7 +129,9 @@ static_assert(B_COUNT <= 16, "mbarrier region holds 16 barriers");
 // TMEM columns (fp32, 128 lanes).  The output and pseudo-value accumulators
 // of a chunk parity are adjacent ([O | U]) so one N = 64 MMA updates both.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t tG0 = 0, tG1 = 384, tOU = 64, tW = 192, tDS = 256;  // tO(p) = tOU + 64 p, tU(p) = tO(p) + 32
+constexpr uint32_t tG0 = 0, tG1 = 384, tW = 192, tDS = 256;
+// [O | U] of chunk t in slot t mod 3: tO = tOU(slot), tU = tO + 32
+__device__ __forceinline__ uint32_t tOU(int slot) { return slot == 2 ? 448u : 64u + 64u * (uint32_t)slot; }
 
 // Launch modes.  kModeChain: one CTA per (b, h) chain over all T tokens.
 // In-device context parallelism (the report's section 5.1.1 SM-level CP,
@@ -143,7 +151,7 @@ struct TcParams {
   float *hT;
   unsigned *status;
   const float *sin;  // [BH][nseg][128][128] entering states (kModeSegFinal)
-  float *m_out;      // [BH][nseg-1][128][128] segment transitions (kModeSegTransition)
+  float *m_out;      // [BH][nseg-1][128][128] segment transitions, transposed (kModeSegTransition)
   float *st_out;     // [BH][nseg-1][128][128] segment states from zero (kModeSegTransition)
   int T;
   int seg_len;
@@ -178,66 +186,98 @@ __device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity
 // hi/lo pair of (a, b): returns packed hi, writes packed lo.
 __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  const float2 r = __ffma2_rn(__bfloat1622float2(h), make_float2(-1.f, -1.f), make_float2(a, b));  // exact residual
+  const __nv_bfloat162 l = __float22bfloat162_rn(r);
   lo = *reinterpret_cast<const uint32_t *>(&l);
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 // ---- token A: decay and rescaled operands of one chunk, 128 threads ----------
 // Thread tt owns the key-channel pair (2pp, 2pp+1) for the 16 tokens of half
-// hf of the chunk.  The token loops are kept rolled: three warpgroups share
-// each SM sub-partition's instruction cache, so code size costs time here.
+// hf of the chunk, in one pass: the first half runs backwards from token 15
+// (x_s = -(g_{s+1} + ... + g_15) >= 0), the second forwards from token 16
+// (x_s = g_16 + ... + g_s <= 0).  Tokens go in groups of four whose shared
+// memory loads are issued before the previous group's stores, so the loop
+// stays rolled (three warpgroups share each sub-partition's instruction
+// cache) without serialising on load latency.
+__device__ __forceinline__ void decay_group(const uint32_t (&gr)[4], const uint32_t (&qr)[4], const uint32_t (&kr)[4],
+                                            float2 &R, bool fwd, unsigned char *qkw, unsigned char *kc,
+                                            const uint32_t (&off)[4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gr[u]));
+    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr[u]));
+    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr[u]));
+    const float2 Rn = __fadd2_rn(R, g);
+    const float2 xr = fwd ? Rn : make_float2(-R.x, -R.y);
+    R = Rn;
+    const float x0 = fminf(fmaxf(xr.x, -87.f), 87.f), x1 = fminf(fmaxf(xr.y, -87.f), 87.f);
+    const float2 ep = make_float2(__expf(x0), __expf(x1)), en = make_float2(__expf(-x0), __expf(-x1));
+    const float2 qe = __fmul2_rn(q, ep), ke = __fmul2_rn(k, ep), ki = __fmul2_rn(k, en);
+    uint32_t qlo, clo;
+    const uint32_t qhi = split2(qe.x, qe.y, qlo);
+    const __nv_bfloat162 khi = __float22bfloat162_rn(ke);
+    const uint32_t chi = split2(ki.x, ki.y, clo);
+    *reinterpret_cast<__nv_bfloat162 *>(qkw + off[u]) = khi;
+    *reinterpret_cast<uint32_t *>(qkw + 4096 + off[u]) = qlo;
+    *reinterpret_cast<uint32_t *>(qkw + 8192 + off[u]) = qhi;
+    *reinterpret_cast<uint32_t *>(kc + off[u]) = chi;
+    *reinterpret_cast<uint32_t *>(kc + 4096 + off[u]) = clo;
+  }
+}
+
 __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs) {
   unsigned char *sm = x.sm;
   const int pp = tt & 63, hf = tt >> 6;
   const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
+  const bool fwd = hf != 0;
   const unsigned char *rg = sm + kRawG + h * 4096;
   const unsigned char *rq = sm + kRawQK + h * 4096;
   const unsigned char *rk = sm + kRawQK + 8192 + h * 4096;
-  // sum of g over the half
-  float S0 = 0.f, S1 = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < 16; ++i) {
-    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rg + sw128_off(16 * hf + i, cc)));
-    S0 += g.x;
-    S1 += g.y;
-  }
-  float *xch = reinterpret_cast<float *>(sm + kXch);
-  *reinterpret_cast<float2 *>(xch + 128 * hf + c0) = make_float2(S0, S1);
-  // tokens 0..15: x = G_s - G_15 (>= 0); tokens 16..31: x = sum_{16..s} g (<= 0)
-  const float b0 = hf == 0 ? S0 : 0.f, b1 = hf == 0 ? S1 : 0.f;
   unsigned char *qkw = sm + kQKW + p * 32768 + h * 16384;  // Ks | Qs lo | Qs | -W~
-  unsigned char *kc = sm + kKC + p * 16384 + h * 8192;     // Kc hi | Kc lo
-  float P0 = 0.f, P1 = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t off = sw128_off(16 * hf + i, cc);
-    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rg + off));
-    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rq + off));
-    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rk + off));
-    P0 += g.x;
-    P1 += g.y;
-    const float x0 = fminf(fmaxf(P0 - b0, -87.f), 87.f), x1 = fminf(fmaxf(P1 - b1, -87.f), 87.f);
-    const float e0 = __expf(x0), e1 = __expf(x1), i0 = __expf(-x0), i1 = __expf(-x1);
-    uint32_t qlo, clo;
-    const uint32_t qhi = split2(q.x * e0, q.y * e1, qlo);
-    const __nv_bfloat162 khi = __floats2bfloat162_rn(k.x * e0, k.y * e1);
-    const uint32_t chi = split2(k.x * i0, k.y * i1, clo);
-    *reinterpret_cast<__nv_bfloat162 *>(qkw + off) = khi;
-    *reinterpret_cast<uint32_t *>(qkw + 4096 + off) = qlo;
-    *reinterpret_cast<uint32_t *>(qkw + 8192 + off) = qhi;
-    *reinterpret_cast<uint32_t *>(kc + off) = chi;
-    *reinterpret_cast<uint32_t *>(kc + 4096 + off) = clo;
+  unsigned char *kc = sm + kKC + fs * 16384 + h * 8192;    // Kc hi | Kc lo
+  // token of step i: 16 + i forwards, 15 - i backwards
+  auto row = [&](int i) { return fwd ? 16 + i : 15 - i; };
+  uint32_t g0[4], q0[4], k0[4], o0[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    o0[u] = sw128_off(row(u), cc);
+    g0[u] = *reinterpret_cast<const uint32_t *>(rg + o0[u]);
+    q0[u] = *reinterpret_cast<const uint32_t *>(rq + o0[u]);
+    k0[u] = *reinterpret_cast<const uint32_t *>(rk + o0[u]);
   }
+  float2 R = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int grp = 0; grp < 4; ++grp) {
+    uint32_t g1[4], q1[4], k1[4], o1[4];
+    if (grp < 3) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        o1[u] = sw128_off(row(4 * grp + 4 + u), cc);
+        g1[u] = *reinterpret_cast<const uint32_t *>(rg + o1[u]);
+        q1[u] = *reinterpret_cast<const uint32_t *>(rq + o1[u]);
+        k1[u] = *reinterpret_cast<const uint32_t *>(rk + o1[u]);
+      }
+    }
+    decay_group(g0, q0, k0, R, fwd, qkw, kc, o0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      g0[u] = g1[u];
+      q0[u] = q1[u];
+      k0[u] = k1[u];
+      o0[u] = o1[u];
+    }
+  }
+  // R = sum of g over the half: rho = G_15 for the first, G_31 - rho for the second
+  float *xch = reinterpret_cast<float *>(sm + kXch);
+  *reinterpret_cast<float2 *>(xch + 128 * hf + c0) = R;
   named_sync(kBarTokA, 128);
   {
     const int c = tt;
-    float *fac = reinterpret_cast<float *>(sm + kFac + fs * 1536);
+    float *fac = reinterpret_cast<float *>(sm + kFac + fs * 1024);
     const float rho = xch[c], tail = xch[128 + c];
     fac[c] = __expf(rho);                // e^rho
-    fac[128 + c] = __expf(rho + tail);   // e^{G_31}
-    fac[256 + c] = __expf(tail);         // e^{G_31 - rho}
+    fac[128 + c] = __expf(tail);         // e^{G_31 - rho}
   }
 }
 
@@ -258,8 +298,9 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt, const float *b
 #pragma unroll
       for (int s = 0; s < r; ++s) acc -= L[(b0 + r) * 33 + b0 + s] * n[s];
       n[r] = acc;
-      N[(b0 + r) * 33 + b0 + jj] = acc;
     }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) N[(b0 + r) * 33 + b0 + jj] = n[r];  // stores after all loads
   }
   named_sync(kBarTokB, 128);
   // level 2: N_10 = -N_11 L_10 N_00 inside each 16x16 block (8x8 pieces)
@@ -280,22 +321,30 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt, const float *b
   }
   named_sync(kBarTokB, 128);
   // level 3: N_10 = -N_11 L_10 N_00 for the two 16x16 blocks (2 elements per thread)
+  {
+    float acc[2];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
-    float acc = 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+      acc[u] = 0.f;
 #pragma unroll
-    for (int s = 0; s < 16; ++s) acc += L[(16 + r) * 33 + s] * N[s * 33 + j];
-    X[r * 17 + j] = acc;
+      for (int s = 0; s < 16; ++s) acc[u] += L[(16 + r) * 33 + s] * N[s * 33 + j];
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) X[((tt + 128 * u) >> 4) * 17 + ((tt + 128 * u) & 15)] = acc[u];
   }
   named_sync(kBarTokB, 128);
+  {
+    float acc[2];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int e = tt + 128 * u, r = e >> 4, j = e & 15;
-    float acc = 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const int e = tt + 128 * u, r = e >> 4, j = e & 15;
+      acc[u] = 0.f;
 #pragma unroll
-    for (int s = 0; s < 16; ++s) acc += N[(16 + r) * 33 + 16 + s] * X[s * 17 + j];
-    N[(16 + r) * 33 + j] = -acc;
+      for (int s = 0; s < 16; ++s) acc[u] += N[(16 + r) * 33 + 16 + s] * X[s * 17 + j];
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) N[(16 + ((tt + 128 * u) >> 4)) * 33 + ((tt + 128 * u) & 15)] = -acc[u];
   }
   named_sync(kBarTokB, 128);
   // T = N Diag(beta), lower triangle, bf16: thread -> (row r, 8-column chunk k)
@@ -314,22 +363,17 @@ __device__ __forceinline__ void token_solve(const Ctx &x, int tt, const float *b
   }
 }
 
-// Row e of S~^T = (Diag(e^rho) S)^T for the 32 channels [32 q, 32 q + 32):
-// four 16-byte chunks of bf16 in the SW128 K-major layout of the S~^T operand.
-__device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const float *__restrict__ erho,
-                                           const float (&S)[D], int e, int q) {
-  float4 r[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) r[i] = reinterpret_cast<const float4 *>(erho + 32 * q)[i];
+// Row e of S~^T for the 32 channels [32 q, 32 q + 32): four 16-byte chunks of
+// bf16 in the SW128 K-major layout of the S~^T operand.
+__device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const float2 (&S)[D / 2], int e, int q) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int c = 32 * q + 8 * k;
-    const float4 a = r[2 * k], b = r[2 * k + 1];
     uint4 w;
-    w.x = pack_bf16x2(a.x * S[c + 0], a.y * S[c + 1]);
-    w.y = pack_bf16x2(a.z * S[c + 2], a.w * S[c + 3]);
-    w.z = pack_bf16x2(b.x * S[c + 4], b.y * S[c + 5]);
-    w.w = pack_bf16x2(b.z * S[c + 6], b.w * S[c + 7]);
+    w.x = pack_bf16x2(S[c / 2 + 0].x, S[c / 2 + 0].y);
+    w.y = pack_bf16x2(S[c / 2 + 1].x, S[c / 2 + 1].y);
+    w.z = pack_bf16x2(S[c / 2 + 2].x, S[c / 2 + 2].y);
+    w.w = pack_bf16x2(S[c / 2 + 3].x, S[c / 2 + 3].y);
     *reinterpret_cast<uint4 *>(st + (q >> 1) * 16384 + sw128_chunk(e, (q & 1) * 4 + k)) = w;
   }
 }
@@ -404,9 +448,13 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t idOU = idesc_bf16(128, 64, false, false, false);
     const uint32_t idS = idesc_bf16(128, 128, false, true, false);
     unsigned char *st = sm + kST;
-    float S[D];
+    // S[i] = rows (2i, 2i+1) of column e: channel pairs, updated with packed f32x2 arithmetic
+    float2 S[D / 2];
 #pragma unroll
-    for (int c = 0; c < D; ++c) S[c] = h0src ? h0src[c * D + e] : (kind == 2 && c == e ? 1.f : 0.f);
+    for (int i = 0; i < D / 2; ++i) {
+      S[i].x = h0src ? h0src[(2 * i) * D + e] : (kind == 2 && 2 * i == e ? 1.f : 0.f);
+      S[i].y = h0src ? h0src[(2 * i + 1) * D + e] : (kind == 2 && 2 * i + 1 == e ? 1.f : 0.f);
+    }
     // [O(t) | V~(t)] = S~^T [Qs; -W~]^T + [0 | U(t)]; called by all of warp 0.  The
     // first K-step is split so O starts from zero while V~ accumulates onto U.
     auto issue_v1 = [&](int t) {
@@ -414,7 +462,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       const uint64_t dS = sdesc_sw128(sbase + kST, 16, 1024);
       const uint64_t dB = sdesc_sw128(sbase + kQKW + pb * 32768 + 8192, 16, 1024);  // rows: Qs, -W~
-      const uint32_t tO = tbase + tOU + 64 * pb;
+      const uint32_t tO = tbase + tOU(t % 3);
       mma_bf16_warp(tO, dS, dB, idO, false);
       mma_bf16_warp(tO + 32, dS, sdesc_add(dB, 4096), idO, true);
 #pragma unroll
@@ -423,12 +471,18 @@ __global__ void __launch_bounds__(NT, 1)
         mma_bf16_warp(tO, sdesc_add(dS, koff), sdesc_add(dB, koff), idOU, true);
       }
       mma_commit_warp(&x.bar[B_V1]);
+      // these MMAs are the last readers of the chunk's double-buffered operands
+      // (Qs, -W~); the triple-buffered ones (Kc, A, factors, [O | U]) are
+      // two chunks behind, so the buffers of parity pb may take chunk t + 2
+      mma_commit_warp(&x.bar[B_CD0 + pb]);
     };
     if (nchunks > 0) {
       const bool ready = wait_bar(x, B_WT0, 0u);
-      const float *erho = reinterpret_cast<const float *>(sm + kFac);
+      const float2 *erho = reinterpret_cast<const float2 *>(sm + kFac);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) store_st32(st, erho, S, e, q);
+      for (int i = 0; i < D / 2; ++i) S[i] = __fmul2_rn(erho[i], S[i]);  // S~ of the first chunk
+#pragma unroll
+      for (int q = 0; q < 4; ++q) store_st32(st, S, e, q);
       fence_proxy_async_smem();
       tc_fence_before();
       named_sync(kBarChain, 128);
@@ -442,7 +496,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       {
         float v[32];
-        tmem_ld32(tl + tOU + 64 * pb + 32, v);
+        tmem_ld32(tl + tOU(t % 3) + 32, v);
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -461,8 +515,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (warp == 0 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
         tc_fence_after();
         const uint64_t dVh = sdesc_sw64(sbase + kVTH, 16, 512), dVl = sdesc_sw64(sbase + kVTL, 16, 512);
-        const uint64_t dKh = sdesc_sw128(sbase + kKC + pb * 16384, 8192, 1024), dKl = sdesc_add(dKh, 4096);
-        const uint64_t dAh = sdesc_sw64(sbase + kAH + pb * 4096, 16, 512), dAl = sdesc_add(dAh, 2048);
+        const uint64_t dKh = sdesc_sw128(sbase + kKC + (t % 3) * 16384, 8192, 1024), dKl = sdesc_add(dKh, 4096);
+        const uint64_t dAh = sdesc_sw64(sbase + kAH + (t % 3) * 4096, 16, 512), dAl = sdesc_add(dAh, 2048);
 #pragma unroll
         for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
           const uint64_t aB = part == 1 ? dVl : dVh;
@@ -472,19 +526,21 @@ __global__ void __launch_bounds__(NT, 1)
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = sdesc_add(aB, ks * 32);
             mma_bf16_warp(tbase + tDS, ad, sdesc_add(kB, ks * 2048), idS, part > 0 || ks > 0);
-            mma_bf16_warp(tbase + tOU + 64 * pb, ad, sdesc_add(mB, ks * 32), idO, true);
+            mma_bf16_warp(tbase + tOU(t % 3), ad, sdesc_add(mB, ks * 32), idO, true);
           }
         }
         mma_commit_warp(&x.bar[B_DS]);
-        // once these MMAs have read them, chunk t's operand buffers may take chunk t + 2
-        mma_commit_warp(&x.bar[B_CD0 + pb]);
       }
       // the next chunk's e^rho (written by token A) is needed to form S~^T(t+1)
       if (has_next) wait_bar(x, B_DEC0 + (pb ^ 1), (uint32_t)((t + 1) >> 1) & 1u);
       wait_bar(x, B_DS, (uint32_t)t & 1u);
       tc_fence_after();
       {
-        const float *fac = reinterpret_cast<const float *>(sm + kFac + (t % 3) * 1536);
+        // S~(t+1) = e^{rho(t+1)} (e^{G_31 - rho} (S~ + dS)), after the last chunk S
+        // itself = e^{G_31 - rho} (S~ + dS).  The two factors stay separate: each is
+        // >= e^-80, their product may underflow fp32 while the result does not.
+        const float *f = reinterpret_cast<const float *>(sm + kFac + (t % 3) * 1024) + 128;
+        const float *fn = reinterpret_cast<const float *>(sm + kFac + ((t + 1) % 3) * 1024);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float ds[32];
@@ -492,21 +548,18 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 a = reinterpret_cast<const float4 *>(fac + 128 + 32 * q4)[i4];
-            const float4 b = reinterpret_cast<const float4 *>(fac + 256 + 32 * q4)[i4];
+            const float4 a = reinterpret_cast<const float4 *>(f + 32 * q4)[i4];
+            const float4 b = has_next ? reinterpret_cast<const float4 *>(fn + 32 * q4)[i4] : make_float4(1.f, 1.f, 1.f, 1.f);
             const int c = 32 * q4 + 4 * i4;
-            S[c + 0] = a.x * S[c + 0] + b.x * ds[4 * i4 + 0];
-            S[c + 1] = a.y * S[c + 1] + b.y * ds[4 * i4 + 1];
-            S[c + 2] = a.z * S[c + 2] + b.z * ds[4 * i4 + 2];
-            S[c + 3] = a.w * S[c + 3] + b.w * ds[4 * i4 + 3];
+            S[c / 2] = __fmul2_rn(make_float2(b.x, b.y),
+                                  __fmul2_rn(make_float2(a.x, a.y), __fadd2_rn(S[c / 2], make_float2(ds[4 * i4 + 0], ds[4 * i4 + 1]))));
+            S[c / 2 + 1] = __fmul2_rn(
+                make_float2(b.z, b.w),
+                __fmul2_rn(make_float2(a.z, a.w), __fadd2_rn(S[c / 2 + 1], make_float2(ds[4 * i4 + 2], ds[4 * i4 + 3]))));
           }
+          if (has_next) store_st32(st, S, e, q4);
         }
-      }
-      if (has_next) {
-        const float *erho = reinterpret_cast<const float *>(sm + kFac + ((t + 1) % 3) * 1536);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) store_st32(st, erho, S, e, q);
-        fence_proxy_async_smem();
+        if (has_next) fence_proxy_async_smem();
       }
       tc_fence_before();
       const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
@@ -523,7 +576,7 @@ __global__ void __launch_bounds__(NT, 1)
       // (rows past the end of the sequence are clipped by the tensor map)
       if (store_o) {
         float ov[32];
-        tmem_ld32(tl + tOU + 64 * pb, ov);
+        tmem_ld32(tl + tOU(t % 3), ov);
         tmem_ld_wait();
         unsigned char *ot = sm + kOst + (e >> 6) * 4096;
 #pragma unroll
@@ -543,9 +596,17 @@ __global__ void __launch_bounds__(NT, 1)
       if (!go) break;
     }
     if (warp == 0 && lane == 0) bulk_wait_all();
-    if (*x.abort == 0 && hdst) {
+    if (*x.abort == 0 && hdst && kind == 2) {
+      // the segment transition is stored transposed (row e = column e of M) for the scan
+      float4 *row = reinterpret_cast<float4 *>(hdst + (size_t)e * D);
 #pragma unroll
-      for (int c = 0; c < D; ++c) hdst[c * D + e] = S[c];
+      for (int i = 0; i < D / 4; ++i) row[i] = make_float4(S[2 * i].x, S[2 * i].y, S[2 * i + 1].x, S[2 * i + 1].y);
+    } else if (*x.abort == 0 && hdst) {
+#pragma unroll
+      for (int i = 0; i < D / 2; ++i) {
+        hdst[(2 * i) * D + e] = S[i].x;
+        hdst[(2 * i + 1) * D + e] = S[i].y;
+      }
     }
   } else if (warp < 8) {
     // ======================= token A (warps 4-7) =======================
@@ -555,16 +616,25 @@ __global__ void __launch_bounds__(NT, 1)
     const unsigned short *beta_bits = reinterpret_cast<const unsigned short *>(beta);
     const uint32_t idG = idesc_bf16(128, 64, false, false, false);
     // TMA issue, called by all of warp 4 (one elected lane issues).
+    // transition runs write no outputs and need no q: its buffer stays zero
+    const bool need_q = store_o;
     auto tma_qkg = [&](int t) {
-      mbar_arrive_expect_tx_warp(&x.bar[B_QKG], 6 * 4096);
+      mbar_arrive_expect_tx_warp(&x.bar[B_QKG], (need_q ? 6 : 4) * 4096);
       const int y = tb + t * C;
-      tma_load_3d_warp(sm + kRawQK, &mq, &x.bar[B_QKG], 0, y, bh);
-      tma_load_3d_warp(sm + kRawQK + 4096, &mq, &x.bar[B_QKG], 64, y, bh);
+      if (need_q) {
+        tma_load_3d_warp(sm + kRawQK, &mq, &x.bar[B_QKG], 0, y, bh);
+        tma_load_3d_warp(sm + kRawQK + 4096, &mq, &x.bar[B_QKG], 64, y, bh);
+      }
       tma_load_3d_warp(sm + kRawQK + 8192, &mk, &x.bar[B_QKG], 0, y, bh);
       tma_load_3d_warp(sm + kRawQK + 12288, &mk, &x.bar[B_QKG], 64, y, bh);
       tma_load_3d_warp(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
       tma_load_3d_warp(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
     };
+    if (!need_q) {
+      uint4 *zq = reinterpret_cast<uint4 *>(sm + kRawQK);
+      for (int i = tt; i < 512; i += 128) zq[i] = make_uint4(0, 0, 0, 0);
+      named_sync(kBarTokA, 128);
+    }
     int qkg_issued = -1;  // last chunk whose q, k, g copy was issued (abort path)
     if (warp == 4 && nchunks > 0) {
       if (lane == 0) {
@@ -594,7 +664,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_after();
         // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
         const uint64_t dA = sdesc_sw128(sbase + kQKW + pb * 32768, 16, 1024);
-        const uint64_t dB = sdesc_sw128(sbase + kKC + pb * 16384, 16, 1024);
+        const uint64_t dB = sdesc_sw128(sbase + kKC + (t % 3) * 16384, 16, 1024);
         const uint32_t tg = tbase + (pb ? tG1 : tG0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
@@ -677,7 +747,9 @@ __global__ void __launch_bounds__(NT, 1)
       named_sync(kBarTokB, 128);
       if (quarter == 2) {
         const float *Xa = reinterpret_cast<const float *>(sm + kXa);
-        unsigned char *ah = sm + kAH + pb * 4096;
+        unsigned char *ah = sm + kAH + (t % 3) * 4096;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a[j] += Xa[r * 33 + j];  // all loads ahead of the stores
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           uint4 hi, lo;
@@ -685,7 +757,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int j = 8 * k + i;
-            m[i] = (j <= r) ? a[j] + Xa[r * 33 + j] : 0.f;
+            m[i] = (j <= r) ? a[j] : 0.f;
           }
           hi.x = split2(m[0], m[1], lo.x);
           hi.y = split2(m[2], m[3], lo.y);
@@ -708,7 +780,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t bd = sdesc_add(dT, ks * 32);
-            mma_bf16_warp(tbase + tOU + 64 * pb + 32, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
+            mma_bf16_warp(tbase + tOU(t % 3) + 32, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
             mma_bf16_warp(tbase + tW, sdesc_add(dKs, ks * 2048), bd, idMK, ks > 0);
           }
           mma_commit_warp(&x.bar[B_UW]);
@@ -760,40 +832,46 @@ __global__ void __launch_bounds__(NT, 1)
 // Entering states of the segments, column block by column block:
 // S_in(0) = h0 (or 0); S_in(s+1) = M_s S_in(s) + S~_s  (Eq. 17's prefix scan).
 // Grid (B*H, 8): each CTA owns 16 state columns of one chain; fp32 throughout.
-__global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const float *M, const float *St, float *Sin,
+// The transitions arrive transposed (MT[k][i] = M[i][k]), so a warp reading
+// M[i][k] for 16 consecutive rows i touches 16 consecutive words; the next
+// transition is loaded into registers while the current one is applied.
+__global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const float *MT, const float *St, float *Sin,
                                                       int nseg) {
   extern __shared__ float cps[];
-  float *Ms = cps;               // [128][129]
-  float *X = cps + 128 * 129;    // [128][16]
+  float *Ms = cps;               // [128 k][128 i]
+  float *X = cps + D * D;        // [128][16]
   const int bh = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
   const int i = tid >> 1, j0 = 8 * (tid & 1);
   const size_t mat = (size_t)D * D;
+  float4 pre[16], spre[2];
+  auto fetch = [&](int s) {
+    const float4 *Mg = reinterpret_cast<const float4 *>(MT + ((size_t)bh * (nseg - 1) + s) * mat);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) pre[u] = __ldg(Mg + tid + 256 * u);
+    const float4 *Sg = reinterpret_cast<const float4 *>(St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0);
+    spre[0] = __ldg(Sg);
+    spre[1] = __ldg(Sg + 1);
+  };
+  if (nseg > 1) fetch(0);
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = h0 ? h0[bh * mat + (size_t)i * D + c0 + j0 + j] : 0.f;
   for (int s = 0;; ++s) {
-    float *out = Sin + ((size_t)bh * nseg + s) * mat + (size_t)i * D + c0 + j0;
+    float4 *out = reinterpret_cast<float4 *>(Sin + ((size_t)bh * nseg + s) * mat + (size_t)i * D + c0 + j0);
+    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      out[j] = acc[j];
-      X[i * 16 + j0 + j] = acc[j];
-    }
+    for (int j = 0; j < 8; ++j) X[i * 16 + j0 + j] = acc[j];
     if (s + 1 >= nseg) break;
-    const float *Mg = M + ((size_t)bh * (nseg - 1) + s) * mat;
-    for (int e = tid; e < D * D / 4; e += 256) {
-      const float4 m4 = reinterpret_cast<const float4 *>(Mg)[e];
-      const int r = (4 * e) / D, c = (4 * e) % D;
-      Ms[r * 129 + c] = m4.x;
-      Ms[r * 129 + c + 1] = m4.y;
-      Ms[r * 129 + c + 2] = m4.z;
-      Ms[r * 129 + c + 3] = m4.w;
-    }
-    __syncthreads();
-    const float *Sg = St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = Sg[j];
+    for (int u = 0; u < 16; ++u) reinterpret_cast<float4 *>(Ms)[tid + 256 * u] = pre[u];
+    acc[0] = spre[0].x, acc[1] = spre[0].y, acc[2] = spre[0].z, acc[3] = spre[0].w;
+    acc[4] = spre[1].x, acc[5] = spre[1].y, acc[6] = spre[1].z, acc[7] = spre[1].w;
+    __syncthreads();
+    if (s + 2 < nseg) fetch(s + 1);
+#pragma unroll 8
     for (int k = 0; k < D; ++k) {
-      const float m = Ms[i * 129 + k];
+      const float m = Ms[k * D + i];
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[j] += m * X[k * 16 + j0 + j];
     }
@@ -875,7 +953,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.mode = kModeSegTransition;
   chunk_tc_kernel<<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int scan_smem = (128 * 129 + 128 * 16) * (int)sizeof(float);
+  const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
     return e;
   cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, P);

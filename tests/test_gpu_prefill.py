@@ -66,6 +66,21 @@ def test_fast_decay_heads_both_paths():
         assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"], chunk
 
 
+@pytest.mark.parametrize("T", [300, 1100])
+def test_decay_at_the_bound(T):
+    # g = g_min = -5 on every token of half the key channels: each 16-token
+    # window there sums to exactly -80, the widest range one reference point
+    # per 32-token chunk has to carry (T = 1100 also runs the segmented path)
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=4, T=T, seed=5)
+    x = synth.prefill_inputs(w)
+    g = x["g"].clone()
+    g[..., :64] = -5.0
+    x["g"] = g
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("B,H,T", [(1, 16, 2305), (1, 2, 2304), (2, 3, 1100), (1, 74, 600)])
 def test_in_device_context_parallel(B, H, T):
     # few chains and enough tokens: the call splits every chain into segments
