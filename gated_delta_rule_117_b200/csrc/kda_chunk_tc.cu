@@ -184,12 +184,15 @@ __device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity
 }
 
 // hi/lo pair of (a, b): returns packed hi, writes packed lo.
+// hi = a, b truncated to bf16 (their upper 16 bits, no conversion needed);
+// lo = the exact residuals rounded to bf16, so hi + lo carries ~16 bits.
 __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float2 r = __ffma2_rn(__bfloat1622float2(h), make_float2(-1.f, -1.f), make_float2(a, b));  // exact residual
+  const uint32_t ua = __float_as_uint(a) & 0xffff0000u, ub = __float_as_uint(b) & 0xffff0000u;
+  const float2 r = __ffma2_rn(make_float2(__uint_as_float(ua), __uint_as_float(ub)), make_float2(-1.f, -1.f),
+                              make_float2(a, b));  // exact residual
   const __nv_bfloat162 l = __float22bfloat162_rn(r);
   lo = *reinterpret_cast<const uint32_t *>(&l);
-  return *reinterpret_cast<const uint32_t *>(&h);
+  return __byte_perm(ua, ub, 0x7632);  // bf16 pair: a in the low half, b in the high half
 }
 
 // ---- token A: decay and rescaled operands of one chunk, 128 threads ----------
@@ -636,7 +639,7 @@ __global__ void __launch_bounds__(NT, 1)
       named_sync(kBarTokA, 128);
     }
     int qkg_issued = -1;  // last chunk whose q, k, g copy was issued (abort path)
-    if (warp == 4 && nchunks > 0) {
+    if (warp == 5 && nchunks > 0) {
       if (lane == 0) {
         prefetch_tmap(&mq);
         prefetch_tmap(&mk);
@@ -660,6 +663,12 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       const bool go = named_sync_and(kBarTokA, 128, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_DEC0 + pb]);
+      // raw q, k, g buffers are free once the decay has read them: warp 5
+      // refills them while warp 4 issues the Gram MMAs
+      if (warp == 5 && __shfl_sync(0xffffffffu, go, 0) && t + 1 < nchunks) {
+        tma_qkg(t + 1);
+        qkg_issued = t + 1;
+      }
       if (warp == 4 && __shfl_sync(0xffffffffu, landed && go, 0)) {
         tc_fence_after();
         // rows [Ks; Qs lo; Qs; -W~ (unused)] x [Kc hi | Kc lo], one N = 64 product
@@ -671,15 +680,11 @@ __global__ void __launch_bounds__(NT, 1)
           mma_bf16_warp(tg, sdesc_add(dA, (ks >> 2) * 16384 + (ks & 3) * 32),
                         sdesc_add(dB, (ks >> 2) * 8192 + (ks & 3) * 32), idG, ks > 0);
         mma_commit_warp(&x.bar[B_GRAM0 + pb]);
-        if (t + 1 < nchunks) {  // raw q, k, g buffers are free once the decay stage has read them
-          tma_qkg(t + 1);
-          qkg_issued = t + 1;
-        }
       }
       beta_cur = beta_next;
       if (!go) break;
     }
-    if (tt == 0 && *x.abort && qkg_issued >= 0)  // let the last q, k, g copy land before the CTA exits
+    if (tt == 32 && *x.abort && qkg_issued >= 0)  // let the last q, k, g copy land before the CTA exits
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_QKG], (uint32_t)qkg_issued & 1u); ++i) {
       }
   } else {
