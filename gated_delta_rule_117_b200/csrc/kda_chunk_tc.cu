@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(NT, 1)
       {
         float v[32];
         tmem_ld32(tl + tOU(t % 3) + 32, v);
-        tmem_ld_wait();
+        tmem_ld_wait(v);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           uint4 hi, lo;
@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int q4 = 0; q4 < 4; ++q4) {
           float ds[32];
           tmem_ld32(tl + tDS + 32 * q4, ds);
-          tmem_ld_wait();
+          tmem_ld_wait(ds);
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
             const float4 a = reinterpret_cast<const float4 *>(f + 32 * q4)[i4];
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (store_o) {
         float ov[32];
         tmem_ld32(tl + tOU(t % 3), ov);
-        tmem_ld_wait();
+        tmem_ld_wait(ov);
         unsigned char *ot = sm + kOst + (e >> 6) * 4096;
 #pragma unroll
         for (int r = 0; r < C; ++r)
@@ -732,7 +732,8 @@ __global__ void __launch_bounds__(NT, 1)
         float b[32];
         tmem_ld32(tl + tg, a);
         tmem_ld32(tl + tg + 32, b);
-        tmem_ld_wait();
+        tmem_ld_wait(a);
+        tmem_ld_touch(b);
 #pragma unroll
         for (int j = 0; j < 32; ++j) a[j] += b[j];
         if (quarter == 0) {
@@ -743,7 +744,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
       } else if (quarter == 1) {
         tmem_ld32(tl + tg, a);
-        tmem_ld_wait();
+        tmem_ld_wait(a);
         float *Xa = reinterpret_cast<float *>(sm + kXa);
 #pragma unroll
         for (int j = 0; j < 32; ++j) Xa[r * 33 + j] = a[j];
@@ -801,7 +802,7 @@ __global__ void __launch_bounds__(NT, 1)
         // -W~[r][c] (K-major rows r) right after Qs in the chunk's operand block
         float w[32];
         tmem_ld32(tl + tW, w);
-        tmem_ld_wait();
+        tmem_ld_wait(w);
         const int c = tt, h = c >> 6, cc = c & 63;
         unsigned char *nw = sm + kQKW + pb * 32768 + h * 16384 + 12288;
 #pragma unroll

@@ -166,6 +166,19 @@ __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Mark the destination registers of a tcgen05.ld as written at this point, so
+// that no use of them is scheduled above the preceding wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_touch(float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+// Wait for this thread's tcgen05.ld copies; `v` is the array they filled.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(float (&v)[N]) {
+  tmem_ld_wait();
+  tmem_ld_touch(v);
+}
 
 // ---- tcgen05.mma (kind::f16: bf16 x bf16 -> fp32 in TMEM) ------------------------
 // Instruction descriptor: D fp32, A/B bf16, dense, K-major (0) or MN-major (1)
