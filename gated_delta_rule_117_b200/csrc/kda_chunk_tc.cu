@@ -169,18 +169,32 @@ struct Ctx {
 
 // Bounded wait: sleeps on the barrier (no spinning), returns false as soon as
 // another role aborted, and gives up after 2 s of wall time.
-__device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity) {
-  uint64_t *b = &x.bar[slot];
-  if (mbar_try_wait(b, parity)) return true;
+__device__ __forceinline__ bool wait_bar_loop(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status) {
   const uint64_t t_start = global_ns();
   for (;;) {
     if (mbar_try_wait_sleep(b, parity, 1000000u)) return true;
-    if (*x.abort) return false;
+    if (*abort) return false;
     if (global_ns() - t_start > 2000000000ull) break;
   }
-  *x.abort = 1;
-  atomicExch(x.status, kDevTimeout);
+  *abort = 1;
+  atomicExch(status, kDevTimeout);
   return false;
+}
+__device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity) {
+  uint64_t *b = &x.bar[slot];
+  if (mbar_try_wait(b, parity)) return true;
+  return wait_bar_loop(b, parity, x.abort, x.status);
+}
+// The token warpgroups share one out-of-line copy of the sleeping loop (their
+// instruction streams compete for each sub-partition's instruction cache).  The
+// chain cannot call: a call inside its 248-register region fails allocation.
+__device__ __noinline__ bool wait_bar_slow(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status) {
+  return wait_bar_loop(b, parity, abort, status);
+}
+__device__ __forceinline__ bool wait_tok(const Ctx &x, int slot, uint32_t parity) {
+  uint64_t *b = &x.bar[slot];
+  if (mbar_try_wait(b, parity)) return true;
+  return wait_bar_slow(b, parity, x.abort, x.status);
 }
 
 // hi/lo pair of (a, b): returns packed hi, writes packed lo.
@@ -285,27 +299,33 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs)
 }
 
 // N = (I + L)^-1 for the strictly lower 32x32 L in Lf (fp32), blocked 8 -> 16 -> 32,
-// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]).  Token B, 128 threads.
+// then T = N Diag(beta) in bf16 (SW64 K-major [r][s]); token B.
+// Level 1: the four 8x8 diagonal blocks of N, one column per lane; run by the
+// warp that wrote L (lanes 0-31), right after it, so it overlaps the A epilogue.
+__device__ __forceinline__ void solve_diag_blocks(const Ctx &x, int lane) {
+  unsigned char *sm = x.sm;
+  const float *L = reinterpret_cast<const float *>(sm + kLf);
+  float *N = reinterpret_cast<float *>(sm + kNf);
+  const int q = lane >> 3, jj = lane & 7, b0 = 8 * q;
+  float n[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    float acc = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+    for (int s = 0; s < r; ++s) acc -= L[(b0 + r) * 33 + b0 + s] * n[s];
+    n[r] = acc;
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) N[(b0 + r) * 33 + b0 + jj] = n[r];  // stores after all loads
+}
+
+// Levels 2 and 3 (128 threads) on the diagonal blocks left by solve_diag_blocks
+// (made visible by a preceding barrier), then T.
 __device__ __forceinline__ void token_solve(const Ctx &x, int tt, const float *bet) {
   unsigned char *sm = x.sm;
   const float *L = reinterpret_cast<const float *>(sm + kLf);
   float *N = reinterpret_cast<float *>(sm + kNf);
   float *X = reinterpret_cast<float *>(sm + kXf);
-  // level 1: the four 8x8 diagonal blocks, one column per thread
-  if (tt < 32) {
-    const int q = tt >> 3, jj = tt & 7, b0 = 8 * q;
-    float n[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float acc = (r == jj) ? 1.f : 0.f;
-#pragma unroll
-      for (int s = 0; s < r; ++s) acc -= L[(b0 + r) * 33 + b0 + s] * n[s];
-      n[r] = acc;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) N[(b0 + r) * 33 + b0 + jj] = n[r];  // stores after all loads
-  }
-  named_sync(kBarTokB, 128);
   // level 2: N_10 = -N_11 L_10 N_00 inside each 16x16 block (8x8 pieces)
   {
     const int blk = tt >> 6, e = tt & 63, r = e >> 3, j = e & 7, o = 16 * blk;
@@ -468,8 +488,8 @@ __global__ void __launch_bounds__(NT, 1)
       const uint32_t tO = tbase + tOU(t % 3);
       mma_bf16_warp(tO, dS, dB, idO, false);
       mma_bf16_warp(tO + 32, dS, sdesc_add(dB, 4096), idO, true);
-#pragma unroll
-      for (int ks = 1; ks < 8; ++ks) {
+#pragma unroll 1
+      for (int ks = 1; ks < 8; ++ks) {  // rolled: MMA issue loops are kept small for the instruction cache
         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
         mma_bf16_warp(tO, sdesc_add(dS, koff), sdesc_add(dB, koff), idOU, true);
       }
@@ -520,7 +540,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint64_t dVh = sdesc_sw64(sbase + kVTH, 16, 512), dVl = sdesc_sw64(sbase + kVTL, 16, 512);
         const uint64_t dKh = sdesc_sw128(sbase + kKC + (t % 3) * 16384, 8192, 1024), dKl = sdesc_add(dKh, 4096);
         const uint64_t dAh = sdesc_sw64(sbase + kAH + (t % 3) * 4096, 16, 512), dAl = sdesc_add(dAh, 2048);
-#pragma unroll
+#pragma unroll 1
         for (int part = 0; part < 3; ++part) {  // V~ hi*hi, lo*hi, hi*lo against Kc and A
           const uint64_t aB = part == 1 ? dVl : dVh;
           const uint64_t kB = part == 2 ? dKl : dKh;
@@ -656,8 +676,8 @@ __global__ void __launch_bounds__(NT, 1)
       const int pb = t & 1, t0 = tb + t * C;
       unsigned short beta_next = 0;
       if (tt < C && t0 + C + tt < te) beta_next = __ldg(beta_bits + t0 + C + tt);
-      if (t >= 2) wait_bar(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);  // chunk t-2's buffers are free
-      const bool landed = wait_bar(x, B_QKG, (uint32_t)t & 1u);
+      if (t >= 2) wait_tok(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);  // chunk t-2's buffers are free
+      const bool landed = wait_tok(x, B_QKG, (uint32_t)t & 1u);
       if (tt < C) reinterpret_cast<float *>(sm + kBeta + pb * 128)[tt] = __bfloat162float(__ushort_as_bfloat16(beta_cur));
       token_decay(x, tt, pb, t % 3);
       fence_proxy_async_smem();
@@ -675,7 +695,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint64_t dA = sdesc_sw128(sbase + kQKW + pb * 32768, 16, 1024);
         const uint64_t dB = sdesc_sw128(sbase + kKC + (t % 3) * 16384, 16, 1024);
         const uint32_t tg = tbase + (pb ? tG1 : tG0);
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks)
           mma_bf16_warp(tg, sdesc_add(dA, (ks >> 2) * 16384 + (ks & 3) * 32),
                         sdesc_add(dB, (ks >> 2) * 8192 + (ks & 3) * 32), idG, ks > 0);
@@ -720,8 +740,8 @@ __global__ void __launch_bounds__(NT, 1)
     for (int t = 0; t < nchunks; ++t) {
       const int pb = t & 1;
       const float *bet = reinterpret_cast<const float *>(sm + kBeta + pb * 128);
-      wait_bar(x, B_DEC0 + pb, (uint32_t)(t >> 1) & 1u);
-      wait_bar(x, B_GRAM0 + pb, (uint32_t)(t >> 1) & 1u);
+      wait_tok(x, B_DEC0 + pb, (uint32_t)(t >> 1) & 1u);
+      wait_tok(x, B_GRAM0 + pb, (uint32_t)(t >> 1) & 1u);
       tc_fence_after();
       // Gram tile -> L (lanes 0-31: Ks rows) and A (lanes 64-95: Qs rows, plus
       // the Qs-lo part from lanes 32-63)
@@ -741,6 +761,8 @@ __global__ void __launch_bounds__(NT, 1)
           float *Lm = reinterpret_cast<float *>(sm + kLf);
 #pragma unroll
           for (int j = 0; j < 32; ++j) Lm[r * 33 + j] = (j < r) ? br * a[j] : 0.f;
+          __syncwarp();
+          solve_diag_blocks(x, lane);
         }
       } else if (quarter == 1) {
         tmem_ld32(tl + tg, a);
@@ -777,7 +799,7 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       named_sync(kBarTokB, 128);
       if (warp == 8 && __shfl_sync(0xffffffffu, !*x.abort, 0)) {
-        const bool vok = v_zero || wait_bar(x, B_V, (uint32_t)t & 1u);
+        const bool vok = v_zero || wait_tok(x, B_V, (uint32_t)t & 1u);
         if (__shfl_sync(0xffffffffu, vok, 0)) {
           tc_fence_after();
           const uint64_t dT = sdesc_sw64(sbase + kTT, 16, 512);
@@ -792,7 +814,7 @@ __global__ void __launch_bounds__(NT, 1)
           mma_commit_warp(&x.bar[B_UW]);
         }
       }
-      const bool uw = wait_bar(x, B_UW, (uint32_t)t & 1u);
+      const bool uw = wait_tok(x, B_UW, (uint32_t)t & 1u);
       tc_fence_after();
       if (warp == 8 && __shfl_sync(0xffffffffu, uw, 0) && t + 1 < nchunks) {  // the U MMA has consumed v
         tma_v(t + 1);
@@ -878,8 +900,10 @@ __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const flo
 #pragma unroll 8
     for (int k = 0; k < D; ++k) {
       const float m = Ms[k * D + i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] += m * X[k * 16 + j0 + j];
+      const float4 xa = *reinterpret_cast<const float4 *>(X + k * 16 + j0);
+      const float4 xb = *reinterpret_cast<const float4 *>(X + k * 16 + j0 + 4);
+      acc[0] += m * xa.x, acc[1] += m * xa.y, acc[2] += m * xa.z, acc[3] += m * xa.w;
+      acc[4] += m * xb.x, acc[5] += m * xb.y, acc[6] += m * xb.z, acc[7] += m * xb.w;
     }
     __syncthreads();
   }
