@@ -875,42 +875,51 @@ __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const flo
   float *Ms = cps;               // [128 k][128 i]
   float *X = cps + D * D;        // [128][16]
   const int bh = blockIdx.x, c0 = 16 * blockIdx.y, tid = threadIdx.x;
-  const int i = tid >> 1, j0 = 8 * (tid & 1);
+  // thread: rows i, i + 1 and columns j0 .. j0 + 3 of the CTA's 16
+  const int i = 2 * (tid >> 2), j0 = 4 * (tid & 3);
   const size_t mat = (size_t)D * D;
   float4 pre[16], spre[2];
   auto fetch = [&](int s) {
     const float4 *Mg = reinterpret_cast<const float4 *>(MT + ((size_t)bh * (nseg - 1) + s) * mat);
 #pragma unroll
     for (int u = 0; u < 16; ++u) pre[u] = __ldg(Mg + tid + 256 * u);
-    const float4 *Sg = reinterpret_cast<const float4 *>(St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0);
-    spre[0] = __ldg(Sg);
-    spre[1] = __ldg(Sg + 1);
+    const float *Sg = St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0;
+    spre[0] = __ldg(reinterpret_cast<const float4 *>(Sg));
+    spre[1] = __ldg(reinterpret_cast<const float4 *>(Sg + D));
   };
   if (nseg > 1) fetch(0);
-  float acc[8];
+  float4 acc[2];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = h0 ? h0[bh * mat + (size_t)i * D + c0 + j0 + j] : 0.f;
+  for (int r = 0; r < 2; ++r)
+    acc[r] = h0 ? *reinterpret_cast<const float4 *>(h0 + bh * mat + (size_t)(i + r) * D + c0 + j0)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0;; ++s) {
-    float4 *out = reinterpret_cast<float4 *>(Sin + ((size_t)bh * nseg + s) * mat + (size_t)i * D + c0 + j0);
-    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    float *out = Sin + ((size_t)bh * nseg + s) * mat + (size_t)i * D + c0 + j0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) X[i * 16 + j0 + j] = acc[j];
+    for (int r = 0; r < 2; ++r) {
+      *reinterpret_cast<float4 *>(out + r * D) = acc[r];
+      *reinterpret_cast<float4 *>(X + (i + r) * 16 + j0) = acc[r];
+    }
     if (s + 1 >= nseg) break;
 #pragma unroll
     for (int u = 0; u < 16; ++u) reinterpret_cast<float4 *>(Ms)[tid + 256 * u] = pre[u];
-    acc[0] = spre[0].x, acc[1] = spre[0].y, acc[2] = spre[0].z, acc[3] = spre[0].w;
-    acc[4] = spre[1].x, acc[5] = spre[1].y, acc[6] = spre[1].z, acc[7] = spre[1].w;
+    // packed accumulators: (row, columns 0-1) and (row, columns 2-3)
+    float2 a00 = make_float2(spre[0].x, spre[0].y), a01 = make_float2(spre[0].z, spre[0].w);
+    float2 a10 = make_float2(spre[1].x, spre[1].y), a11 = make_float2(spre[1].z, spre[1].w);
     __syncthreads();
     if (s + 2 < nseg) fetch(s + 1);
 #pragma unroll 8
     for (int k = 0; k < D; ++k) {
-      const float m = Ms[k * D + i];
-      const float4 xa = *reinterpret_cast<const float4 *>(X + k * 16 + j0);
-      const float4 xb = *reinterpret_cast<const float4 *>(X + k * 16 + j0 + 4);
-      acc[0] += m * xa.x, acc[1] += m * xa.y, acc[2] += m * xa.z, acc[3] += m * xa.w;
-      acc[4] += m * xb.x, acc[5] += m * xb.y, acc[6] += m * xb.z, acc[7] += m * xb.w;
+      const float2 m = *reinterpret_cast<const float2 *>(Ms + k * D + i);  // M[i][k], M[i+1][k]
+      const float4 xv = *reinterpret_cast<const float4 *>(X + k * 16 + j0);
+      const float2 xlo = make_float2(xv.x, xv.y), xhi = make_float2(xv.z, xv.w);
+      a00 = __ffma2_rn(make_float2(m.x, m.x), xlo, a00);
+      a01 = __ffma2_rn(make_float2(m.x, m.x), xhi, a01);
+      a10 = __ffma2_rn(make_float2(m.y, m.y), xlo, a10);
+      a11 = __ffma2_rn(make_float2(m.y, m.y), xhi, a11);
     }
+    acc[0] = make_float4(a00.x, a00.y, a01.x, a01.y);
+    acc[1] = make_float4(a10.x, a10.y, a11.x, a11.y);
     __syncthreads();
   }
 }
