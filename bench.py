@@ -274,7 +274,8 @@ def main():
     trec = traffic_record("%s:%s" % (kernel_name, w.name), src)
     traffic = None
     if trec:
-        traffic = trec["dram_bytes_per_launch"]
+        # a segmented step records the DRAM bytes of all its launches, like `achieved`
+        traffic = trec.get("dram_bytes_per_step", trec.get("dram_bytes_per_launch"))
 
     e2e = measure_e2e(args, w, x, kda, torch, dev, plan)
 
