@@ -297,6 +297,8 @@ def main():
         "e2e": e2e,
         "gpu_launches": plan["launches"] * args.steps,
     }
+    if world == 1 and T >= CKPT_INTERVAL:
+        result["ckpt"] = measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step)
     if not args.no_decode and world == 1:
         result["decode"] = measure_decode(args, synth, kda, torch, dev, pk, pk_kind)
     clocks = clk.summary()
@@ -312,6 +314,44 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result))
+
+
+CKPT_INTERVAL = 512  # hash-block size of the prefix cache (tokens)
+
+
+def measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, plain_ms):
+    """The same step through kda_chunk_fwd_ckpt, persisting the state every
+    CKPT_INTERVAL tokens for a prefix cache: time per step and its overhead."""
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+    dev, sp = o.device, torch.cuda.current_stream().cuda_stream
+    n = T // CKPT_INTERVAL
+    ck = torch.empty(B, H, n, dk, dv, dtype=torch.float32, device=dev)
+    dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
+    ptr = lambda t: None if t is None else t.data_ptr()
+
+    def step():
+        st = kda.kda_chunk_fwd_ckpt(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["g"]), ptr(d["beta"]), ptr(h0),
+                                    ptr(o), ptr(hT), ck.data_ptr(), CKPT_INTERVAL, B, H, T, dk, dv, dt,
+                                    args.chunk_size, 0.0, ws.data_ptr(), ws.numel(), sp)
+        if st != 0:
+            raise kda.KdaError(st, "kda_chunk_fwd_ckpt")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
+    return {"interval": CKPT_INTERVAL, "checkpoints_per_chain": n, "ms_per_step": ms,
+            "overhead": ms / plain_ms - 1.0, "extra_bytes_per_step": B * H * n * dk * dv * 4,
+            "gpu_launches": len(ev) * launches}
 
 
 def measure_e2e(args, w, x, kda, torch, dev, plan):

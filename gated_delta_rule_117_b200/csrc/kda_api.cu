@@ -117,18 +117,25 @@ size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dty
   return p.workspace;
 }
 
-kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
-                           const void *beta, const float *h0, void *o, float *h_T, int B, int H,
-                           int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
-                           void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// kda_chunk_fwd and kda_chunk_fwd_ckpt (ckpt == nullptr: no checkpoints).
+kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                       const float *h0, void *o, float *h_T, float *ckpt, int ckpt_interval, int B, int H,
+                       int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream) {
   kda_plan_t plan;
   kda_status_t st = plan_prefill(B, H, T, dk, dv, dtype, chunk_size, &plan);
   if (st != KDA_OK) return st;
   if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  const int n_ckpt = ckpt_interval > 0 ? T / ckpt_interval : 0;
   if (B * H == 0) return KDA_OK;
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+  if (n_ckpt > 0 && !ckpt) return KDA_ERR_INVALID_ARG;
   const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
-  const void *ptrs[] = {q, k, v, g, h0, o, h_T, workspace};
+  const void *ptrs[] = {q, k, v, g, h0, o, h_T, workspace, n_ckpt > 0 ? ckpt : nullptr};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
   if (beta && ((uintptr_t)beta % e) != 0) return KDA_ERR_ALIGNMENT;
@@ -139,7 +146,8 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
               rv = range_of(v, n * T * dv * e), rg = range_of(g, n * T * dk * e),
               rb = range_of(beta, n * T * e), rh0 = range_of(h0, h0 ? n * dk * dv * 4 : 0),
               ro = range_of(o, n * T * dv * e), rhT = range_of(h_T, h_T ? n * dk * dv * 4 : 0),
-              rw = range_of(workspace, plan.workspace);
+              rw = range_of(workspace, plan.workspace),
+              rc = range_of(ckpt, n_ckpt > 0 ? n * n_ckpt * dk * dv * 4 : 0);
   const Range ins[] = {rq, rk, rv, rg, rb, rh0};
   for (const Range &r : ins)
     if (overlap(ro, r)) return KDA_ERR_ALIAS;
@@ -148,8 +156,9 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
   if (h_T && h0 && overlap(rhT, rh0) && (const void *)h_T != (const void *)h0) return KDA_ERR_ALIAS;
   if (overlap(rhT, ro)) return KDA_ERR_ALIAS;
   for (const Range &r : ins)
-    if (overlap(rw, r)) return KDA_ERR_ALIAS;
+    if (overlap(rw, r) || overlap(rc, r)) return KDA_ERR_ALIAS;
   if (overlap(rw, ro) || overlap(rw, rhT)) return KDA_ERR_ALIAS;
+  if (overlap(rc, ro) || overlap(rc, rhT) || overlap(rc, rw)) return KDA_ERR_ALIAS;
 
   st = check_device();
   if (st != KDA_OK) return st;
@@ -162,11 +171,36 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
   a.status = kda::device_status_ptr();
   a.workspace = workspace;
   a.segments = plan.segments;
+  a.ckpt = n_ckpt > 0 ? ckpt : nullptr;
+  a.ckpt_interval = ckpt_interval;
+  a.n_ckpt = n_ckpt;
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
   const cudaError_t ce = plan.path == KDA_PATH_TC32 ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
                                                     : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
   return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
+                           const void *beta, const float *h0, void *o, float *h_T, int B, int H,
+                           int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
+                           void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, nullptr, 0, B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
+                   workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, const float *h0, void *o, float *h_T, float *ckpt,
+                                int ckpt_interval, int B, int H, int T, int dk, int dv,
+                                kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
+                                size_t workspace_bytes, kda_stream_t stream) {
+  if (ckpt_interval <= 0 || ckpt_interval % 64 != 0) return KDA_ERR_INVALID_ARG;
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, T, dk, dv, dtype, chunk_size, scale,
+                   workspace, workspace_bytes, stream);
 }
 
 kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,

@@ -61,7 +61,8 @@ template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(NT, 1)
     chunk16_kernel(const TIn *__restrict__ qg, const TIn *__restrict__ kg, const TIn *__restrict__ vg,
                    const TIn *__restrict__ gg, const TIn *__restrict__ betag,
-                   const float *h0, TIn *__restrict__ og, float *hT, int T, float scale) {
+                   const float *h0, TIn *__restrict__ og, float *hT, int T, float scale, float *ckpt,
+                   int ckpt_interval, int n_ckpt) {
   using L = SimtSmem<DK, DV>;
   constexpr int LK = L::LK;
   constexpr int CPT = DV / 16;  // output columns per thread in (row, column-group) layouts
@@ -205,6 +206,13 @@ __global__ void __launch_bounds__(NT, 1)
       for (int r = 0; r < C; ++r) acc += Kc[r * LK + i] * Vs[r * DV + j];
       S[e] = acc;
     }
+    // state checkpoint at a hash-aligned position (prefix caching)
+    const int pend = t0 + C;
+    if (ckpt && pend <= T && pend % ckpt_interval == 0) {
+      __syncthreads();
+      float *dst = ckpt + (bh * n_ckpt + pend / ckpt_interval - 1) * (size_t)(DK * DV);
+      for (int e = tid; e < DK * DV; e += NT) dst[e] = S[e];
+    }
   }
   __syncthreads();
   if (hT)
@@ -219,7 +227,7 @@ cudaError_t launch_t(const ChunkArgs &a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   kern<<<a.B * a.H, NT, smem, st>>>((const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v,
                                     (const TIn *)a.g, (const TIn *)a.beta, a.h0, (TIn *)a.o, a.hT,
-                                    a.T, a.scale);
+                                    a.T, a.scale, a.ckpt, a.ckpt_interval, a.n_ckpt);
   return cudaGetLastError();
 }
 

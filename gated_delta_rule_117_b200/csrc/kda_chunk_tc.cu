@@ -153,6 +153,9 @@ struct TcParams {
   const float *sin;  // [BH][nseg][128][128] entering states (kModeSegFinal)
   float *m_out;      // [BH][nseg-1][128][128] segment transitions, transposed (kModeSegTransition)
   float *st_out;     // [BH][nseg-1][128][128] segment states from zero (kModeSegTransition)
+  float *ckpt;        // [BH][n_ckpt][128][128] state checkpoints (chain and final modes), or null
+  int ckpt_interval;  // tokens between checkpoints (a multiple of 64)
+  int n_ckpt;
   int T;
   int seg_len;
   int nseg;
@@ -401,6 +404,9 @@ __device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const
   }
 }
 
+// kCkpt: the instantiation that can emit prefix-cache checkpoints; the plain
+// one compiles without that code so its register allocation is untouched.
+template <bool kCkpt>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
@@ -567,6 +573,12 @@ __global__ void __launch_bounds__(NT, 1)
         // >= e^-80, their product may underflow fp32 while the result does not.
         const float *f = reinterpret_cast<const float *>(sm + kFac + (t % 3) * 1024) + 128;
         const float *fn = reinterpret_cast<const float *>(sm + kFac + ((t + 1) % 3) * 1024);
+        // at a hash-aligned chunk end S itself also goes to the checkpoint buffer
+        // (prefix caching): that rare chunk leaves out the next chunk's factor in
+        // the update, stores S, then applies the factor
+        const int pend = t0 + C;
+        const bool ck = kCkpt && p.ckpt && pend <= te && pend % p.ckpt_interval == 0;
+        const bool sn = has_next && !ck;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float ds[32];
@@ -575,7 +587,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
             const float4 a = reinterpret_cast<const float4 *>(f + 32 * q4)[i4];
-            const float4 b = has_next ? reinterpret_cast<const float4 *>(fn + 32 * q4)[i4] : make_float4(1.f, 1.f, 1.f, 1.f);
+            const float4 b = sn ? reinterpret_cast<const float4 *>(fn + 32 * q4)[i4] : make_float4(1.f, 1.f, 1.f, 1.f);
             const int c = 32 * q4 + 4 * i4;
             S[c / 2] = __fmul2_rn(make_float2(b.x, b.y),
                                   __fmul2_rn(make_float2(a.x, a.y), __fadd2_rn(S[c / 2], make_float2(ds[4 * i4 + 0], ds[4 * i4 + 1]))));
@@ -583,7 +595,22 @@ __global__ void __launch_bounds__(NT, 1)
                 make_float2(b.z, b.w),
                 __fmul2_rn(make_float2(a.z, a.w), __fadd2_rn(S[c / 2 + 1], make_float2(ds[4 * i4 + 2], ds[4 * i4 + 3]))));
           }
-          if (has_next) store_st32(st, S, e, q4);
+          if (sn) store_st32(st, S, e, q4);
+        }
+        if (ck) {
+          float *ckp = p.ckpt + ((size_t)bh * p.n_ckpt + pend / p.ckpt_interval - 1) * D * D + e;
+#pragma unroll
+          for (int i = 0; i < D / 2; ++i) {
+            ckp[(size_t)(2 * i) * D] = S[i].x;
+            ckp[(size_t)(2 * i + 1) * D] = S[i].y;
+          }
+          if (has_next) {
+            const float2 *ern = reinterpret_cast<const float2 *>(fn);
+#pragma unroll
+            for (int i = 0; i < D / 2; ++i) S[i] = __fmul2_rn(ern[i], S[i]);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) store_st32(st, S, e, q4);
+          }
         }
         if (has_next) fence_proxy_async_smem();
       }
@@ -974,14 +1001,22 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.m_out = p.st_out = nullptr;
   p.T = a.T;
   p.scale = a.scale;
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  p.ckpt = a.ckpt;
+  p.ckpt_interval = a.ckpt_interval > 0 ? a.ckpt_interval : 1;
+  p.n_ckpt = a.n_ckpt;
+  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int P = a.segments > 1 ? a.segments : 1;
   if (P == 1) {
     p.seg_len = a.T > 0 ? a.T : 1;
     p.nseg = 1;
     p.mode = kModeChain;
-    chunk_tc_kernel<<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    if (p.ckpt)
+      chunk_tc_kernel<true><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    else
+      chunk_tc_kernel<false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();
   }
   const size_t mat = (size_t)D * D;
@@ -996,7 +1031,9 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.st_out = Sw;
   p.sin = Sin;
   p.mode = kModeSegTransition;
-  chunk_tc_kernel<<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  float *const ckpt = p.ckpt;
+  p.ckpt = nullptr;  // transition runs start from 0 or I: no checkpoints there
+  chunk_tc_kernel<false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
@@ -1004,7 +1041,11 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, P);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.mode = kModeSegFinal;
-  chunk_tc_kernel<<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  p.ckpt = ckpt;
+  if (p.ckpt)
+    chunk_tc_kernel<true><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  else
+    chunk_tc_kernel<false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   return cudaGetLastError();
 }
 

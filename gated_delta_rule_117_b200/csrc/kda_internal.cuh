@@ -24,6 +24,9 @@ struct ChunkArgs {
   unsigned *status;
   void *workspace;  // scratch of at least the planned size (context-parallel passes)
   int segments;     // in-device context-parallel segments per chain (1 = none)
+  float *ckpt;        // [B*H][n_ckpt][dk][dv] state checkpoints, or null
+  int ckpt_interval;  // tokens between checkpoints (multiple of 64) when ckpt is set
+  int n_ckpt;         // T / ckpt_interval
 };
 
 struct DecodeArgs {

@@ -24,7 +24,7 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
-            "kda_noalloc_scratch_bytes"]
+            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt"]
 
 
 class KdaError(RuntimeError):
@@ -59,6 +59,8 @@ def load_library():
             lib.kda_chunk_fwd_workspace_size.restype = sz
             lib.kda_chunk_fwd.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
             lib.kda_chunk_fwd.restype = i
+            lib.kda_chunk_fwd_ckpt.argtypes = [vp] * 9 + [i] * 8 + [f, vp, sz, vp]
+            lib.kda_chunk_fwd_ckpt.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
             lib.kda_recurrent_step.restype = i
             lib.kda_status_string.argtypes = [i]
@@ -103,6 +105,14 @@ def kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_si
     """Returns the raw kda_status_t."""
     return load_library().kda_chunk_fwd(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size,
                                         scale, workspace, workspace_bytes, stream)
+
+
+def kda_chunk_fwd_ckpt(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, T, dk, dv, dtype, chunk_size,
+                       scale, workspace, workspace_bytes, stream) -> int:
+    """kda_chunk_fwd that also writes state checkpoints every ckpt_interval tokens.
+    Returns the raw kda_status_t."""
+    return load_library().kda_chunk_fwd_ckpt(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, T, dk, dv,
+                                             dtype, chunk_size, scale, workspace, workspace_bytes, stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
@@ -153,10 +163,13 @@ def _stream(stream):
 
 
 def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, h_T=None, scale=0.0, chunk_size=0,
-              output_final_state=True, workspace=None, stream=None):
+              output_final_state=True, workspace=None, stream=None, ckpt_interval=0, ckpt=None):
     """Prefill over [B, H, T, d] tensors (see kda_chunk_fwd in include/kda.h).
 
-    Allocates o / h_T / workspace with torch when not given.  Returns (o, h_T).
+    Allocates o / h_T / workspace with torch when not given.  Returns (o, h_T),
+    or (o, h_T, ckpt) when ckpt_interval > 0 (kda_chunk_fwd_ckpt: ckpt is
+    [B, H, T // ckpt_interval, dk, dv] fp32, the state at every multiple of
+    ckpt_interval tokens).
     """
     import torch
     B, H, T, dk = q.shape
@@ -171,9 +184,18 @@ def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, h_T=None, scale=0.0, chunk_s
         raise KdaError(2, "kda_chunk_fwd_workspace_size")
     if ws > 0 and workspace is None:
         workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if ckpt_interval:
+        if ckpt is None:
+            ckpt = torch.empty(B, H, T // ckpt_interval, dk, dv, dtype=torch.float32, device=q.device)
+        st = kda_chunk_fwd_ckpt(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(h_T),
+                                _ptr(ckpt), ckpt_interval, B, H, T, dk, dv, dt, chunk_size, float(scale),
+                                _ptr(workspace), wbytes, _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd_ckpt")
+        return o, h_T, ckpt
     st = kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(h_T),
-                       B, H, T, dk, dv, dt, chunk_size, float(scale), _ptr(workspace),
-                       0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+                       B, H, T, dk, dv, dt, chunk_size, float(scale), _ptr(workspace), wbytes, _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
     return o, h_T

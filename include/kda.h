@@ -142,6 +142,30 @@ kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, con
                                 kda_dtype_t dtype, float scale, kda_stream_t stream);
 
 /*
+ * Prefill that also emits recurrent-state checkpoints for prefix caching
+ * (Kimi K3 report, section 5.4.1: after a forward pass the KDA kernel persists
+ * the recurrent state at hash-block-aligned positions, so a later request that
+ * shares the prefix can copy the snapshot and resume prefill at that token).
+ *
+ * Same arguments, layouts, alignment, aliasing rules and results as
+ * kda_chunk_fwd, plus:
+ *   ckpt_interval : hash-block size in tokens; a positive multiple of 64
+ *   ckpt          : [B, H, T / ckpt_interval, dk, dv] fp32 (integer division),
+ *                   16-byte aligned; entry j is the state after token
+ *                   (j + 1) * ckpt_interval - 1, i.e. the state from which
+ *                   prefill resumes at token (j + 1) * ckpt_interval (with that
+ *                   snapshot as h0).  Written, never read.  May be NULL only when
+ *                   T < ckpt_interval (no entry).  Must not overlap any input,
+ *                   o or h_T.
+ * Returns KDA_ERR_INVALID_ARG for a bad interval or a missing buffer.
+ */
+kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, const void *g,
+                                const void *beta, const float *h0, void *o, float *h_T, float *ckpt,
+                                int ckpt_interval, int B, int H, int T, int dk, int dv,
+                                kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
+                                size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

@@ -10,7 +10,10 @@ computes, in fp64:
   update derived from Eq. 1 (numpy, one chain at a time);
 * ``transition``  -- the per-segment pair (cumulative transition M, state from
   zero S~) of KDA Context Parallelism (section 5.1.2, Eq. 17), used to pin the
-  oracle and to check in-device context parallelism.
+  oracle and to check in-device context parallelism;
+* ``checkpoints`` -- the recurrent state at every multiple of a block size,
+  the snapshots section 5.4.1 persists for prefix caching (by definition the
+  final state of each prefix).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It shares no code with the CUDA library
@@ -91,3 +94,22 @@ def recurrent(q, k, v, g, beta, h0=None, scale=None, erase=True, nthreads=None):
     if rc != 0:
         raise RuntimeError("oracle failed (%d)" % rc)
     return o, hT
+
+
+def checkpoints(q, k, v, g, beta, h0=None, interval=512, scale=None):
+    """States a prefix cache would persist (Kimi K3 report, section 5.4.1): entry
+    j is the state after token (j + 1) * interval - 1, i.e. h_T of the prefix of
+    (j + 1) * interval tokens, computed here by running the recurrence on that
+    prefix.  Shapes as for ``recurrent``; returns [..., T // interval, dk, dv]."""
+    T = np.shape(q)[-2]
+    out = []
+    for j in range(T // interval):
+        p = (j + 1) * interval
+        _, hT = recurrent(np.asarray(q)[..., :p, :], np.asarray(k)[..., :p, :], np.asarray(v)[..., :p, :],
+                          np.asarray(g)[..., :p, :], np.asarray(beta)[..., :p], h0, scale=scale)
+        out.append(hT)
+    lead = np.shape(q)[:-2]
+    dk, dv = np.shape(q)[-1], np.shape(v)[-1]
+    if not out:
+        return np.zeros(lead + (0, dk, dv))
+    return np.stack(out, axis=-3)

@@ -95,6 +95,34 @@ def test_chunk_fwd_empty_batch_is_noop(lib):
     assert _call(B=0) == 0 and _call(H=0, q=None) == 0
 
 
+def _ccall(**over):
+    # kda_chunk_fwd_ckpt: the valid arguments of _call plus a checkpoint buffer past h_T
+    n = N
+    a = dict(q=BASE, k=BASE + n, v=BASE + 2 * n, g=BASE + 3 * n, beta=BASE + 4 * n, h0=BASE + 5 * n,
+             o=BASE + 6 * n, h_T=BASE + 7 * n, ckpt=BASE + 8 * n, ckpt_interval=64, B=1, H=2, T=64, dk=16, dv=16,
+             dtype=0, chunk_size=16, scale=0.0, workspace=None, workspace_bytes=0, stream=None)
+    a.update(over)
+    return kda.kda_chunk_fwd_ckpt(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(ckpt_interval=0), 1), (dict(ckpt_interval=32), 1), (dict(ckpt_interval=100), 1),
+    (dict(ckpt=None), 1),                    # one snapshot due (T = 64) but no buffer
+    (dict(ckpt=BASE + 8 * N + 4), 4),
+    (dict(ckpt=BASE + 7 * N), 5),            # checkpoints overlap h_T
+    (dict(ckpt=BASE + 2 * N), 5),            # checkpoints overlap v
+    (dict(dk=24), 2),
+])
+def test_chunk_fwd_ckpt_rejects(lib, over, code):
+    assert _ccall(**over) == code
+
+
+def test_chunk_fwd_ckpt_needs_no_buffer_without_a_boundary(lib):
+    st = _ccall(ckpt=None, T=63)
+    if not torch.cuda.is_available():
+        assert st in (7, 9)
+
+
 def _dcall(**over):
     B, H, dk, dv = 4, 2, 16, 16
     n = 4096

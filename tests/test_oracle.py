@@ -11,7 +11,10 @@ Each pin is chosen so that a plausible mistake in the oracle fails it:
   * scalar closed form           -- textbook first-order linear recurrence;
   * chunk-size independence      -- the UT transform / chunked restatement;
   * state split                  -- h0 handling and the carried state;
-  * KCP linearity (Eq. 17)       -- S_T(h0) = S~_T + M h0.
+  * KCP linearity (Eq. 17)       -- S_T(h0) = S~_T + M h0;
+  * prefix-cache checkpoints     -- each snapshot is the brute-force state at
+    (section 5.4.1)                 its position, and prefill resumed from a
+                                    snapshot reproduces the rest of the run.
 """
 import math
 import os
@@ -251,3 +254,34 @@ def test_empty_sequence_returns_h0():
     e = np.zeros((0, 3))
     o, hT = oracle.recurrent(e, e, np.zeros((0, 4)), e, np.zeros(0), h0)
     assert o.shape == (0, 4) and np.array_equal(hT, h0)
+
+
+def test_checkpoints_are_brute_force_prefix_states():
+    # section 5.4.1: the snapshot at a block boundary p is the state after token p - 1
+    rs = np.random.default_rng(515)
+    T, dk, dv, interval = 7, 3, 2, 3
+    q, k, v, g, beta = _rand_inputs(rs, T, dk, dv, unit_k=False)
+    h0 = rs.standard_normal((dk, dv))
+    ck = oracle.checkpoints(q, k, v, g, beta, h0, interval=interval, scale=0.5)
+    assert ck.shape == (T // interval, dk, dv)
+    for j in range(T // interval):
+        p = (j + 1) * interval
+        _, S_p = _brute(q[:p], k[:p], v[:p], g[:p], beta[:p], h0, 0.5)
+        np.testing.assert_allclose(ck[j], S_p, rtol=0, atol=1e-12)
+
+
+def test_resume_from_checkpoint_reproduces_the_run():
+    rs = np.random.default_rng(516)
+    T, dk, dv, interval = 200, 8, 6, 64
+    q, k, v, g, beta = _rand_inputs(rs, T, dk, dv)
+    h0 = 0.02 * rs.standard_normal((dk, dv))
+    o, hT = oracle.recurrent(q, k, v, g, beta, h0)
+    ck = oracle.checkpoints(q, k, v, g, beta, h0, interval=interval)
+    assert ck.shape == (3, dk, dv)
+    for j in range(3):
+        p = (j + 1) * interval
+        o2, h2 = oracle.recurrent(q[p:], k[p:], v[p:], g[p:], beta[p:], ck[j])
+        np.testing.assert_allclose(o2, o[p:], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(h2, hT, rtol=1e-12, atol=1e-13)
+    # no block boundary inside a short sequence: no snapshot
+    assert oracle.checkpoints(q[:50], k[:50], v[:50], g[:50], beta[:50], h0, interval=interval).shape == (0, dk, dv)
