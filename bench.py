@@ -299,6 +299,8 @@ def main():
     }
     if world == 1 and T >= CKPT_INTERVAL:
         result["ckpt"] = measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step)
+    if world == 1 and B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
+        result["gate"] = measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, ms_per_step)
     if not args.no_decode and world == 1:
         result["decode"] = measure_decode(args, synth, kda, torch, dev, pk, pk_kind)
     clocks = clk.summary()
@@ -352,6 +354,42 @@ def measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, plain_ms):
     return {"interval": CKPT_INTERVAL, "checkpoints_per_chain": n, "ms_per_step": ms,
             "overhead": ms / plain_ms - 1.0, "extra_bytes_per_step": B * H * n * dk * dv * 4,
             "gpu_launches": len(ev) * launches}
+
+
+def measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, plain_ms):
+    """The same step through kda_chunk_fwd_gated (Eq. 5 gate fused into the
+    loads: z and A in, g never in memory): time per step against the plain call,
+    and the bytes a separate gate pass would move (read z, write g)."""
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+    gi = synth.gate_inputs(w)
+    z, A = gi["z"].to(o.device), gi["A_log"].to(o.device)
+    dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
+    sp = torch.cuda.current_stream().cuda_stream
+    ptr = lambda t: None if t is None else t.data_ptr()
+
+    def step():
+        st = kda.kda_chunk_fwd_gated(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), z.data_ptr(), A.data_ptr(), -5.0,
+                                     ptr(d["beta"]), ptr(h0), ptr(o), ptr(hT), B, H, T, dk, dv, dt, args.chunk_size,
+                                     0.0, ws.data_ptr(), ws.numel(), sp)
+        if st != 0:
+            raise kda.KdaError(st, "kda_chunk_fwd_gated")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
+    e = 2 if w.dtype == "bf16" else 4
+    return {"ms_per_step": ms, "overhead": ms / plain_ms - 1.0,
+            "separate_gate_bytes_per_step": 2 * B * H * T * dk * e, "gpu_launches": len(ev) * launches}
 
 
 def measure_e2e(args, w, x, kda, torch, dev, plan):

@@ -122,10 +122,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dty
 namespace {
 
 // kda_chunk_fwd and kda_chunk_fwd_ckpt (ckpt == nullptr: no checkpoints).
+// g holds the logits z when A_log is set (fused Eq. 5 gate).
 kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
-                       const float *h0, void *o, float *h_T, float *ckpt, int ckpt_interval, int B, int H,
-                       int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
-                       size_t workspace_bytes, kda_stream_t stream) {
+                       const float *h0, void *o, float *h_T, float *ckpt, int ckpt_interval, const float *A_log,
+                       float g_min, int B, int H, int T, int dk, int dv, kda_dtype_t dtype, int chunk_size,
+                       float scale, void *workspace, size_t workspace_bytes, kda_stream_t stream) {
   kda_plan_t plan;
   kda_status_t st = plan_prefill(B, H, T, dk, dv, dtype, chunk_size, &plan);
   if (st != KDA_OK) return st;
@@ -134,6 +135,7 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
   if (B * H == 0) return KDA_OK;
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
   if (n_ckpt > 0 && !ckpt) return KDA_ERR_INVALID_ARG;
+  if (A_log && ((uintptr_t)A_log & 3u) != 0) return KDA_ERR_ALIGNMENT;
   const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
   const void *ptrs[] = {q, k, v, g, h0, o, h_T, workspace, n_ckpt > 0 ? ckpt : nullptr};
   for (const void *p : ptrs)
@@ -159,6 +161,8 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
     if (overlap(rw, r) || overlap(rc, r)) return KDA_ERR_ALIAS;
   if (overlap(rw, ro) || overlap(rw, rhT)) return KDA_ERR_ALIAS;
   if (overlap(rc, ro) || overlap(rc, rhT) || overlap(rc, rw)) return KDA_ERR_ALIAS;
+  const Range ra = range_of(A_log, A_log ? (size_t)H * dk * 4 : 0);
+  if (overlap(ra, ro) || overlap(ra, rhT) || overlap(ra, rw) || overlap(ra, rc)) return KDA_ERR_ALIAS;
 
   st = check_device();
   if (st != KDA_OK) return st;
@@ -174,6 +178,8 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
   a.ckpt = n_ckpt > 0 ? ckpt : nullptr;
   a.ckpt_interval = ckpt_interval;
   a.n_ckpt = n_ckpt;
+  a.A_log = A_log;
+  a.g_min = g_min;
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
   const cudaError_t ce = plan.path == KDA_PATH_TC32 ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
@@ -189,8 +195,8 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
                            const void *beta, const float *h0, void *o, float *h_T, int B, int H,
                            int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
                            void *workspace, size_t workspace_bytes, kda_stream_t stream) {
-  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, nullptr, 0, B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
-                   workspace_bytes, stream);
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, nullptr, 0, nullptr, 0.f, B, H, T, dk, dv, dtype, chunk_size, scale,
+                   workspace, workspace_bytes, stream);
 }
 
 kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, const void *g,
@@ -199,7 +205,18 @@ kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, con
                                 kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
                                 size_t workspace_bytes, kda_stream_t stream) {
   if (ckpt_interval <= 0 || ckpt_interval % 64 != 0) return KDA_ERR_INVALID_ARG;
-  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, T, dk, dv, dtype, chunk_size, scale,
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, nullptr, 0.f, B, H, T, dk, dv, dtype,
+                   chunk_size, scale, workspace, workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *z,
+                                 const float *A_log, float g_min, const void *beta, const float *h0,
+                                 void *o, float *h_T, int B, int H, int T, int dk, int dv,
+                                 kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
+                                 size_t workspace_bytes, kda_stream_t stream) {
+  if (!(g_min >= -5.f && g_min < 0.f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
+  if (B > 0 && H > 0 && T > 0 && !A_log) return KDA_ERR_INVALID_ARG;
+  return chunk_fwd(q, k, v, z, beta, h0, o, h_T, nullptr, 0, A_log, g_min, B, H, T, dk, dv, dtype, chunk_size, scale,
                    workspace, workspace_bytes, stream);
 }
 

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(NT, 1)
     chunk16_kernel(const TIn *__restrict__ qg, const TIn *__restrict__ kg, const TIn *__restrict__ vg,
                    const TIn *__restrict__ gg, const TIn *__restrict__ betag,
                    const float *h0, TIn *__restrict__ og, float *hT, int T, float scale, float *ckpt,
-                   int ckpt_interval, int n_ckpt) {
+                   int ckpt_interval, int n_ckpt, const float *A_log, float g_min, int H) {
   using L = SimtSmem<DK, DV>;
   constexpr int LK = L::LK;
   constexpr int CPT = DV / 16;  // output columns per thread in (row, column-group) layouts
@@ -93,7 +93,10 @@ __global__ void __launch_bounds__(NT, 1)
       const size_t off = (size_t)(t0 + r) * DK + c;
       Qe[r * LK + c] = ok ? ld_f(q + off) : 0.f;
       Kn[r * LK + c] = ok ? ld_f(k + off) : 0.f;
-      Kc[r * LK + c] = ok ? ld_f(g + off) : 0.f;  // raw g for the cumsum
+      float gv = ok ? ld_f(g + off) : 0.f;  // raw g for the cumsum
+      if (A_log && ok)  // fused Eq. 5 gate: the input holds the logits z
+        gv = g_min / (1.f + expf(-expf(A_log[(bh % H) * DK + c]) * gv));
+      Kc[r * LK + c] = gv;
     }
     for (int e = tid; e < C * DV; e += NT) {
       const int r = e / DV, c = e % DV;
@@ -227,7 +230,7 @@ cudaError_t launch_t(const ChunkArgs &a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   kern<<<a.B * a.H, NT, smem, st>>>((const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v,
                                     (const TIn *)a.g, (const TIn *)a.beta, a.h0, (TIn *)a.o, a.hT,
-                                    a.T, a.scale, a.ckpt, a.ckpt_interval, a.n_ckpt);
+                                    a.T, a.scale, a.ckpt, a.ckpt_interval, a.n_ckpt, a.A_log, a.g_min, a.H);
   return cudaGetLastError();
 }
 

@@ -156,6 +156,9 @@ struct TcParams {
   float *ckpt;        // [BH][n_ckpt][128][128] state checkpoints (chain and final modes), or null
   int ckpt_interval;  // tokens between checkpoints (a multiple of 64)
   int n_ckpt;
+  const float *A_log;  // [H][128] decay log-scales of the fused Eq. 5 gate (the g map then holds z)
+  float g_min;
+  int H;
   int T;
   int seg_len;
   int nseg;
@@ -220,12 +223,19 @@ __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
 // memory loads are issued before the previous group's stores, so the loop
 // stays rolled (three warpgroups share each sub-partition's instruction
 // cache) without serialising on load latency.
+template <bool kGate>
 __device__ __forceinline__ void decay_group(const uint32_t (&gr)[4], const uint32_t (&qr)[4], const uint32_t (&kr)[4],
                                             float2 &R, bool fwd, unsigned char *qkw, unsigned char *kc,
-                                            const uint32_t (&off)[4]) {
+                                            const uint32_t (&off)[4], float2 eA, float g_min, int row0, int nvalid) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gr[u]));
+    float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gr[u]));
+    if (kGate) {  // the loaded values are the logits z: g = g_min Sigmoid(e^A z)  (Eq. 5)
+      const float2 t = __fmul2_rn(eA, g);
+      g = make_float2(__fdividef(g_min, 1.f + __expf(-t.x)), __fdividef(g_min, 1.f + __expf(-t.y)));
+      // rows past the end of the sequence (zero-filled z) must not decay: g = 0 there
+      if ((fwd ? row0 + u : row0 - u) >= nvalid) g = make_float2(0.f, 0.f);
+    }
     const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr[u]));
     const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr[u]));
     const float2 Rn = __fadd2_rn(R, g);
@@ -246,7 +256,8 @@ __device__ __forceinline__ void decay_group(const uint32_t (&gr)[4], const uint3
   }
 }
 
-__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs) {
+template <bool kGate>
+__device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs, float2 eA, float g_min, int nvalid) {
   unsigned char *sm = x.sm;
   const int pp = tt & 63, hf = tt >> 6;
   const int c0 = 2 * pp, h = c0 >> 6, cc = c0 & 63;
@@ -279,7 +290,7 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs)
         k1[u] = *reinterpret_cast<const uint32_t *>(rk + o1[u]);
       }
     }
-    decay_group(g0, q0, k0, R, fwd, qkw, kc, o0);
+    decay_group<kGate>(g0, q0, k0, R, fwd, qkw, kc, o0, eA, g_min, row(4 * grp), nvalid);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       g0[u] = g1[u];
@@ -404,9 +415,10 @@ __device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const
   }
 }
 
-// kCkpt: the instantiation that can emit prefix-cache checkpoints; the plain
-// one compiles without that code so its register allocation is untouched.
-template <bool kCkpt>
+// kCkpt: the instantiation that can emit prefix-cache checkpoints; kGate: the
+// one whose g input holds the Eq. 5 logits z.  The plain one compiles without
+// either, so its register allocation is untouched.
+template <bool kCkpt, bool kGate>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
@@ -670,6 +682,12 @@ __global__ void __launch_bounds__(NT, 1)
     const int tt = tid - 128;
     const __nv_bfloat16 *beta = p.beta + (size_t)bh * T;
     const unsigned short *beta_bits = reinterpret_cast<const unsigned short *>(beta);
+    // this thread's key-channel pair (see token_decay): e^A of the fused gate
+    float2 eA = make_float2(1.f, 1.f);
+    if (kGate) {
+      const float *Ah = p.A_log + (size_t)(bh % p.H) * D + 2 * (tt & 63);
+      eA = make_float2(__expf(Ah[0]), __expf(Ah[1]));
+    }
     const uint32_t idG = idesc_bf16(128, 64, false, false, false);
     // TMA issue, called by all of warp 4 (one elected lane issues).
     // transition runs write no outputs and need no q: its buffer stays zero
@@ -712,7 +730,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (t >= 2) wait_tok(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);  // chunk t-2's buffers are free
       const bool landed = wait_tok(x, B_QKG, (uint32_t)t & 1u);
       if (tt < C) reinterpret_cast<float *>(sm + kBeta + pb * 128)[tt] = __bfloat162float(__ushort_as_bfloat16(beta_cur));
-      token_decay(x, tt, pb, t % 3);
+      token_decay<kGate>(x, tt, pb, t % 3, eA, p.g_min, te - t0);
       fence_proxy_async_smem();
       const bool go = named_sync_and(kBarTokA, 128, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_DEC0 + pb]);
@@ -1004,9 +1022,16 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.ckpt = a.ckpt;
   p.ckpt_interval = a.ckpt_interval > 0 ? a.ckpt_interval : 1;
   p.n_ckpt = a.n_ckpt;
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  p.A_log = a.A_log;
+  p.g_min = a.g_min;
+  p.H = a.H;
+  const bool gated = a.A_log != nullptr;
+  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunk_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunk_tc_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int P = a.segments > 1 ? a.segments : 1;
   if (P == 1) {
@@ -1014,9 +1039,11 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
     p.nseg = 1;
     p.mode = kModeChain;
     if (p.ckpt)
-      chunk_tc_kernel<true><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+      chunk_tc_kernel<true, false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    else if (gated)
+      chunk_tc_kernel<false, true><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
     else
-      chunk_tc_kernel<false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+      chunk_tc_kernel<false, false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();
   }
   const size_t mat = (size_t)D * D;
@@ -1033,7 +1060,10 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.mode = kModeSegTransition;
   float *const ckpt = p.ckpt;
   p.ckpt = nullptr;  // transition runs start from 0 or I: no checkpoints there
-  chunk_tc_kernel<false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  if (gated)
+    chunk_tc_kernel<false, true><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  else
+    chunk_tc_kernel<false, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
@@ -1043,9 +1073,11 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.mode = kModeSegFinal;
   p.ckpt = ckpt;
   if (p.ckpt)
-    chunk_tc_kernel<true><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    chunk_tc_kernel<true, false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  else if (gated)
+    chunk_tc_kernel<false, true><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   else
-    chunk_tc_kernel<false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    chunk_tc_kernel<false, false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
   return cudaGetLastError();
 }
 

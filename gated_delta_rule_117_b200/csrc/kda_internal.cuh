@@ -27,6 +27,8 @@ struct ChunkArgs {
   float *ckpt;        // [B*H][n_ckpt][dk][dv] state checkpoints, or null
   int ckpt_interval;  // tokens between checkpoints (multiple of 64) when ckpt is set
   int n_ckpt;         // T / ckpt_interval
+  const float *A_log;  // [H][dk] decay log-scales when `g` holds the logits z (fused Eq. 5 gate), else null
+  float g_min;         // lower bound of the fused gate
 };
 
 struct DecodeArgs {

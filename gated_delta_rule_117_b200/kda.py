@@ -24,7 +24,7 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
-            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt"]
+            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated"]
 
 
 class KdaError(RuntimeError):
@@ -61,6 +61,8 @@ def load_library():
             lib.kda_chunk_fwd.restype = i
             lib.kda_chunk_fwd_ckpt.argtypes = [vp] * 9 + [i] * 8 + [f, vp, sz, vp]
             lib.kda_chunk_fwd_ckpt.restype = i
+            lib.kda_chunk_fwd_gated.argtypes = [vp] * 5 + [f] + [vp] * 4 + [i] * 7 + [f, vp, sz, vp]
+            lib.kda_chunk_fwd_gated.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
             lib.kda_recurrent_step.restype = i
             lib.kda_status_string.argtypes = [i]
@@ -113,6 +115,14 @@ def kda_chunk_fwd_ckpt(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, 
     Returns the raw kda_status_t."""
     return load_library().kda_chunk_fwd_ckpt(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, B, H, T, dk, dv,
                                              dtype, chunk_size, scale, workspace, workspace_bytes, stream)
+
+
+def kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale,
+                        workspace, workspace_bytes, stream) -> int:
+    """kda_chunk_fwd with the Eq. 5 decay gate fused into the loads (takes the
+    logits z and log-scales A_log instead of g).  Returns the raw kda_status_t."""
+    return load_library().kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk, dv, dtype,
+                                              chunk_size, scale, workspace, workspace_bytes, stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
@@ -198,6 +208,32 @@ def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, h_T=None, scale=0.0, chunk_s
                        B, H, T, dk, dv, dt, chunk_size, float(scale), _ptr(workspace), wbytes, _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
+    return o, h_T
+
+
+def chunk_fwd_gated(q, k, v, z, A_log, beta, h0=None, *, g_min=-5.0, o=None, h_T=None, scale=0.0, chunk_size=0,
+                    output_final_state=True, workspace=None, stream=None):
+    """Prefill with the fused Eq. 5 gate: z [B, H, T, dk] (dtype of q), A_log
+    [H, dk] fp32.  Allocates o / h_T / workspace when not given.  Returns (o, h_T)."""
+    import torch
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_T is None and output_final_state:
+        h_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    ws = kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dt, chunk_size)
+    if ws == (1 << 64) - 1:
+        raise KdaError(2, "kda_chunk_fwd_workspace_size")
+    if ws > 0 and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta), _ptr(h0),
+                             _ptr(o), _ptr(h_T), B, H, T, dk, dv, dt, chunk_size, float(scale), _ptr(workspace),
+                             wbytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_gated")
     return o, h_T
 
 

@@ -125,6 +125,17 @@ def head_inputs(w: Workload, b: int, h: int, T: Optional[int] = None) -> Dict[st
                 g=round_to(g, w.dtype), beta=round_to(beta, w.dtype), h0=h0)
 
 
+def gate_inputs(w: Workload, T: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The decay logits z [B, H, T, dk] (rounded to the workload dtype) and the
+    log-scales A [H, dk] (fp32) behind every workload's g: the raw draws, before
+    any gate arithmetic, for calls that take z and A instead of g."""
+    T = w.T if T is None else T
+    z = np.stack([np.stack([round_to(_rng(w, _Z, b, h).standard_normal((T, w.dk)), w.dtype) for h in range(w.H)])
+                  for b in range(w.B)])
+    A = np.stack([round_to(decay_log_scale(w, h), "f32") for h in range(w.H)])
+    return dict(z=_to_torch(z, w.torch_dtype), A_log=torch.from_numpy(A).float())
+
+
 def head_input_blocks(w: Workload, b: int, h: int, T: Optional[int] = None, block: int = 65536):
     """The stored inputs of one (b, h) chain in token blocks (same values as
     head_inputs: every stream is drawn sequentially).  Yields (t0, dict) with

@@ -166,6 +166,28 @@ kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, con
                                 size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Prefill with the decay gate fused into the loads (Kimi K3 report, section
+ * 2.1.1, Eq. 5): instead of the log-decay g the call takes the decay logits z
+ * and the log-scales A and forms, per token and key channel,
+ *     g = g_min * Sigmoid(exp(A[h][c]) * z[b][h][t][c])
+ * in fp32 on chip, so g never goes through memory.
+ *
+ * Same arguments, layouts, alignment, aliasing rules and results as
+ * kda_chunk_fwd with g replaced by:
+ *   z     : [B, H, T, dk] dtype (16-byte aligned)
+ *   A_log : [H, dk] fp32, 4-byte aligned (a per-head scale is the same value
+ *           repeated over dk); read only
+ *   g_min : the lower bound of the log-decay, in [-5, 0) (the report fixes
+ *           -5; a bound below -5 would break the e^{80} range the chunked
+ *           kernels rely on); otherwise KDA_ERR_INVALID_ARG
+ */
+kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *z,
+                                 const float *A_log, float g_min, const void *beta, const float *h0,
+                                 void *o, float *h_T, int B, int H, int T, int dk, int dv,
+                                 kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
+                                 size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

@@ -11,6 +11,7 @@ computes, in fp64:
 * ``transition``  -- the per-segment pair (cumulative transition M, state from
   zero S~) of KDA Context Parallelism (section 5.1.2, Eq. 17), used to pin the
   oracle and to check in-device context parallelism;
+* ``gate``        -- the lower-bounded decay gate of Eq. 5, g = g_min Sigmoid(e^A z);
 * ``checkpoints`` -- the recurrent state at every multiple of a block size,
   the snapshots section 5.4.1 persists for prefix caching (by definition the
   final state of each prefix).
@@ -113,3 +114,12 @@ def checkpoints(q, k, v, g, beta, h0=None, interval=512, scale=None):
     if not out:
         return np.zeros(lead + (0, dk, dv))
     return np.stack(out, axis=-3)
+
+
+def gate(z, A_log, g_min=-5.0):
+    """Eq. 5 of the Kimi K3 report: the per-channel log-decay
+    g = g_min * Sigmoid(exp(A) * z), in fp64.  z [..., H, T, dk], A_log [H, dk]
+    (broadcast over the leading and token dimensions)."""
+    z = np.asarray(z, dtype=np.float64)
+    eA = np.exp(np.asarray(A_log, dtype=np.float64))[:, None, :]
+    return g_min / (1.0 + np.exp(-eA * z))

@@ -123,6 +123,26 @@ def test_chunk_fwd_ckpt_needs_no_buffer_without_a_boundary(lib):
         assert st in (7, 9)
 
 
+def _gcall(**over):
+    # kda_chunk_fwd_gated: _call's arguments with z in place of g plus A_log after h_T
+    n = N
+    a = dict(q=BASE, k=BASE + n, v=BASE + 2 * n, z=BASE + 3 * n, A_log=BASE + 8 * n, g_min=-5.0, beta=BASE + 4 * n,
+             h0=BASE + 5 * n, o=BASE + 6 * n, h_T=BASE + 7 * n, B=1, H=2, T=64, dk=16, dv=16, dtype=0,
+             chunk_size=16, scale=0.0, workspace=None, workspace_bytes=0, stream=None)
+    a.update(over)
+    return kda.kda_chunk_fwd_gated(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(g_min=-6.0), 1), (dict(g_min=0.0), 1), (dict(g_min=float("nan")), 1), (dict(A_log=None), 1),
+    (dict(A_log=BASE + 8 * N + 2), 4),
+    (dict(A_log=BASE + 6 * N), 5),           # A_log inside o
+    (dict(z=BASE + N + 4), 4),
+])
+def test_chunk_fwd_gated_rejects(lib, over, code):
+    assert _gcall(**over) == code
+
+
 def _dcall(**over):
     B, H, dk, dv = 4, 2, 16, 16
     n = 4096

@@ -12,6 +12,7 @@ Each pin is chosen so that a plausible mistake in the oracle fails it:
   * chunk-size independence      -- the UT transform / chunked restatement;
   * state split                  -- h0 handling and the carried state;
   * KCP linearity (Eq. 17)       -- S_T(h0) = S~_T + M h0;
+  * Eq. 5 gate                   -- midpoint, bounds, limits, per-channel scale;
   * prefix-cache checkpoints     -- each snapshot is the brute-force state at
     (section 5.4.1)                 its position, and prefill resumed from a
                                     snapshot reproduces the rest of the run.
@@ -285,3 +286,23 @@ def test_resume_from_checkpoint_reproduces_the_run():
         np.testing.assert_allclose(h2, hT, rtol=1e-12, atol=1e-13)
     # no block boundary inside a short sequence: no snapshot
     assert oracle.checkpoints(q[:50], k[:50], v[:50], g[:50], beta[:50], h0, interval=interval).shape == (0, dk, dv)
+
+
+def test_gate_eq5_closed_forms():
+    # Eq. 5: g = g_min Sigmoid(e^A z), in (g_min, 0); A is a per-head, per-channel log-scale
+    A = np.array([[0.0, math.log(2.0)], [-1.0, 0.5]])
+    z = np.zeros((1, 2, 1, 2))
+    np.testing.assert_allclose(oracle.gate(z, A), -2.5, rtol=0, atol=1e-15)  # Sigmoid(0) = 1/2
+    z = np.array([[[[1.0, 1.0]], [[-2.0, 3.0]]]])
+    ref = -5.0 / (1.0 + np.exp(-np.array([[[1.0, 2.0]], [[-2.0 * math.exp(-1.0), 3.0 * math.exp(0.5)]]])))
+    np.testing.assert_allclose(oracle.gate(z, A)[0], ref, rtol=1e-15)
+    big = oracle.gate(np.full((1, 2, 1, 2), 200.0), A)
+    small = oracle.gate(np.full((1, 2, 1, 2), -200.0), A)
+    assert np.all(big >= -5.0) and np.all(big < -4.999999) and np.all(small < 0) and np.all(small > -1e-9)
+    zz = np.random.default_rng(5).standard_normal((2, 2, 50, 2)) * 3
+    gg = oracle.gate(zz, A)
+    assert np.all(gg > -5.0) and np.all(gg < 0.0)
+    # retention alpha = e^g stays above e^{g_min} (the bound the report prints)
+    assert np.exp(gg).min() > math.exp(-5.0)
+    # a different g_min scales the gate
+    np.testing.assert_allclose(oracle.gate(zz, A, g_min=-2.0), gg * 0.4, rtol=1e-14)

@@ -104,3 +104,16 @@ def test_block_generation_matches_whole_draw():
     assert [t0 for t0, _ in parts] == [0, 128, 256]
     for name in ("q", "k", "v", "g", "beta"):
         assert np.array_equal(np.concatenate([x[name] for _, x in parts]), whole[name])
+
+
+def test_gate_inputs_are_the_draws_behind_g():
+    # z and A are the raw draws the workload's g comes from: the Eq. 5 gate of
+    # them reproduces g up to the bf16 rounding of z and of g
+    import oracle
+    w = synth.WORKLOADS["batched_b8_h32_t8k"].with_(B=1, H=4, T=64)
+    gi = synth.gate_inputs(w)
+    assert gi["z"].shape == (1, 4, 64, 128) and gi["z"].dtype == torch.bfloat16
+    assert gi["A_log"].shape == (4, 128) and gi["A_log"].dtype == torch.float32
+    g = oracle.gate(gi["z"].double().numpy(), gi["A_log"].double().numpy())
+    x = synth.prefill_inputs(w)
+    assert np.abs(g - x["g"].double().numpy()).max() < 0.05
