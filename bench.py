@@ -299,6 +299,8 @@ def main():
     }
     if world == 1 and T >= CKPT_INTERVAL:
         result["ckpt"] = measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step)
+    if world == 1:
+        result["out_gate"] = measure_out_gate(args, w, o, flush, kda, torch, pk)
     if world == 1 and B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
         result["gate"] = measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, ms_per_step)
     if not args.no_decode and world == 1:
@@ -390,6 +392,39 @@ def measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, plain_ms):
     e = 2 if w.dtype == "bf16" else 4
     return {"ms_per_step": ms, "overhead": ms / plain_ms - 1.0,
             "separate_gate_bytes_per_step": 2 * B * H * T * dk * e, "gpu_launches": len(ev) * launches}
+
+
+def measure_out_gate(args, w, o, flush, kda, torch, pk):
+    """Eq. 6 output edge (per-head RMSNorm and sigmoid gate) on the prefill's
+    output: an HBM-bound pass, reported against the copy bandwidth."""
+    B, H, T, dv = o.shape
+    gen = torch.Generator(device=o.device).manual_seed(7)
+    gate = torch.randn(o.shape, generator=gen, device=o.device).to(o.dtype)
+    wt = torch.ones(H, dv, dtype=torch.float32, device=o.device)
+    y = torch.empty_like(o)
+    dt = kda.KDA_DTYPE_BF16 if o.dtype == torch.bfloat16 else kda.KDA_DTYPE_F32
+    sp = torch.cuda.current_stream().cuda_stream
+
+    def step():
+        st = kda.kda_output_gate(o.data_ptr(), gate.data_ptr(), wt.data_ptr(), 1e-6, y.data_ptr(), B, H, T, dv, dt, sp)
+        if st != 0:
+            raise kda.KdaError(st, "kda_output_gate")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    nbytes = 3 * o.numel() * o.element_size() + wt.numel() * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac_of_hbm_peak": gbs / pk["hbm_gbs"], "gpu_launches": len(ev)}
 
 
 def measure_e2e(args, w, x, kda, torch, dev, plan):

@@ -220,6 +220,34 @@ kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, co
                    workspace, workspace_bytes, stream);
 }
 
+kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_weight, float eps, void *y,
+                             int B, int H, int T, int dv, kda_dtype_t dtype, kda_stream_t stream) {
+  if (B < 0 || H < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (!supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  if (!(eps >= 0.f) || !isfinite(eps)) return KDA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)B * H * T;
+  if (rows == 0) return KDA_OK;
+  if (!o || !gate || !rms_weight || !y) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {o, gate, rms_weight, y};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+  const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+  const Range ro = range_of(o, rows * dv * e), rg = range_of(gate, rows * dv * e),
+              rw = range_of(rms_weight, (size_t)H * dv * 4), ry = range_of(y, rows * dv * e);
+  if (overlap(ry, rg) || overlap(ry, rw)) return KDA_ERR_ALIAS;
+  if (overlap(ry, ro) && y != o) return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  kda::OutGateArgs a;
+  a.o = o; a.gate = gate; a.w = rms_weight; a.y = y;
+  a.B = B; a.H = H; a.T = T; a.dv = dv;
+  a.bf16 = dtype == KDA_DTYPE_BF16;
+  a.eps = eps;
+  return kda::launch_out_gate(a, (cudaStream_t)stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
                                 const void *beta, float *S, void *o, int B, int H, int dk, int dv,
                                 kda_dtype_t dtype, float scale, kda_stream_t stream) {

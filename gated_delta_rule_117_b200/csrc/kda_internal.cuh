@@ -40,6 +40,16 @@ struct DecodeArgs {
   float scale;
 };
 
+struct OutGateArgs {
+  const void *o, *gate;
+  const float *w;  // [H][dv] RMSNorm weights
+  void *y;
+  int B, H, T, dv;
+  int bf16;
+  float eps;
+};
+
+cudaError_t launch_out_gate(const OutGateArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t s);
 // Planning of the tensor-core path: segments per chain, segment length, workspace bytes.

@@ -24,7 +24,7 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
-            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated"]
+            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate"]
 
 
 class KdaError(RuntimeError):
@@ -63,6 +63,8 @@ def load_library():
             lib.kda_chunk_fwd_ckpt.restype = i
             lib.kda_chunk_fwd_gated.argtypes = [vp] * 5 + [f] + [vp] * 4 + [i] * 7 + [f, vp, sz, vp]
             lib.kda_chunk_fwd_gated.restype = i
+            lib.kda_output_gate.argtypes = [vp, vp, vp, f, vp] + [i] * 5 + [vp]
+            lib.kda_output_gate.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
             lib.kda_recurrent_step.restype = i
             lib.kda_status_string.argtypes = [i]
@@ -123,6 +125,11 @@ def kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk,
     logits z and log-scales A_log instead of g).  Returns the raw kda_status_t."""
     return load_library().kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk, dv, dtype,
                                               chunk_size, scale, workspace, workspace_bytes, stream)
+
+
+def kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream) -> int:
+    """Eq. 6 output edge: y = Sigmoid(gate) * RMSNorm(o).  Returns the raw kda_status_t."""
+    return load_library().kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
@@ -235,6 +242,19 @@ def chunk_fwd_gated(q, k, v, z, A_log, beta, h0=None, *, g_min=-5.0, o=None, h_T
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_gated")
     return o, h_T
+
+
+def output_gate(o, gate, rms_weight, eps=1e-6, *, y=None, stream=None):
+    """Eq. 6 output edge over [B, H, T, dv] tensors; rms_weight [H, dv] fp32.  Returns y."""
+    import torch
+    B, H, T, dv = o.shape
+    if y is None:
+        y = torch.empty_like(o)
+    st = kda_output_gate(_ptr(o), _ptr(gate), _ptr(rms_weight), float(eps), _ptr(y), B, H, T, dv, _dtype_code(o),
+                         _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_output_gate")
+    return y
 
 
 def recurrent_step(q, k, v, g, beta, S, *, o=None, scale=0.0, stream=None):

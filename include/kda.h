@@ -188,6 +188,23 @@ kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, co
                                  size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Output edge of a KDA layer (Kimi K3 report, section 2.1.1, Eq. 6): per-head
+ * RMSNorm of the recurrent output followed by the data-dependent sigmoid gate,
+ *     y[b,h,t,:] = Sigmoid(gate[b,h,t,:]) * w[h,:] * o[b,h,t,:] / sqrt(mean(o[b,h,t,:]^2) + eps)
+ * The projections W_g x (giving `gate`, already split into heads) and W_o are
+ * outside the call.
+ *
+ *   o, gate, y : [B, H, T, dv] dtype, 16-byte aligned; y == o (in place) is
+ *                allowed, any other overlap of y with an input is not
+ *   rms_weight : [H, dv] fp32, 16-byte aligned
+ *   eps        : finite, >= 0
+ *   dv         : one of 16, 32, 64, 128
+ * Errors are reported like kda_chunk_fwd's; the call allocates nothing.
+ */
+kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_weight, float eps, void *y,
+                             int B, int H, int T, int dv, kda_dtype_t dtype, kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

@@ -12,6 +12,7 @@ computes, in fp64:
   zero S~) of KDA Context Parallelism (section 5.1.2, Eq. 17), used to pin the
   oracle and to check in-device context parallelism;
 * ``gate``        -- the lower-bounded decay gate of Eq. 5, g = g_min Sigmoid(e^A z);
+* ``output_gate`` -- the output edge of Eq. 6, Sigmoid(gate) * RMSNorm(o);
 * ``checkpoints`` -- the recurrent state at every multiple of a block size,
   the snapshots section 5.4.1 persists for prefix caching (by definition the
   final state of each prefix).
@@ -123,3 +124,14 @@ def gate(z, A_log, g_min=-5.0):
     z = np.asarray(z, dtype=np.float64)
     eA = np.exp(np.asarray(A_log, dtype=np.float64))[:, None, :]
     return g_min / (1.0 + np.exp(-eA * z))
+
+
+def output_gate(o, gate, w, eps=1e-6):
+    """Eq. 6 of the Kimi K3 report without its projections: per-head RMSNorm of
+    the recurrent output (over dv, weights w [H, dv]) times Sigmoid(gate), in
+    fp64.  o, gate [B, H, T, dv]."""
+    o = np.asarray(o, dtype=np.float64)
+    gate = np.asarray(gate, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)[:, None, :]
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    return (1.0 / (1.0 + np.exp(-gate))) * w * o / rms

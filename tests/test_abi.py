@@ -143,6 +143,32 @@ def test_chunk_fwd_gated_rejects(lib, over, code):
     assert _gcall(**over) == code
 
 
+def _ocall(**over):
+    n = 1 * 2 * 64 * 128 * 2  # bytes of one [1, 2, 64, 128] bf16 tensor
+    a = dict(o=BASE, gate=BASE + n, rms_weight=BASE + 2 * n, eps=1e-6, y=BASE + 3 * n, B=1, H=2, T=64, dv=128,
+             dtype=1, stream=None)
+    a.update(over)
+    return kda.kda_output_gate(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(o=None), 1), (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1), (dict(T=-1), 1),
+    (dict(dv=100), 2), (dict(dtype=4), 3),
+    (dict(gate=BASE + 32768 + 8), 4), (dict(rms_weight=BASE + 65536 + 4), 4),
+    (dict(y=BASE + 32768), 5),          # y overlaps gate
+    (dict(y=BASE + 16), 5),             # y partially overlaps o
+])
+def test_output_gate_rejects(lib, over, code):
+    assert _ocall(**over) == code
+
+
+def test_output_gate_in_place_and_empty(lib):
+    assert _ocall(B=0) == 0
+    st = _ocall(y=BASE)  # y == o: in place is allowed
+    if not torch.cuda.is_available():
+        assert st in (7, 9)
+
+
 def _dcall(**over):
     B, H, dk, dv = 4, 2, 16, 16
     n = 4096

@@ -13,6 +13,7 @@ Each pin is chosen so that a plausible mistake in the oracle fails it:
   * state split                  -- h0 handling and the carried state;
   * KCP linearity (Eq. 17)       -- S_T(h0) = S~_T + M h0;
   * Eq. 5 gate                   -- midpoint, bounds, limits, per-channel scale;
+  * Eq. 6 output edge            -- hand-worked row, scale invariance, unit RMS;
   * prefix-cache checkpoints     -- each snapshot is the brute-force state at
     (section 5.4.1)                 its position, and prefill resumed from a
                                     snapshot reproduces the rest of the run.
@@ -306,3 +307,24 @@ def test_gate_eq5_closed_forms():
     assert np.exp(gg).min() > math.exp(-5.0)
     # a different g_min scales the gate
     np.testing.assert_allclose(oracle.gate(zz, A, g_min=-2.0), gg * 0.4, rtol=1e-14)
+
+
+def test_output_gate_eq6():
+    # hand-worked row: o = (3, 4), mean square 12.5, gate 0 -> Sigmoid = 1/2, w = (1, 2)
+    o = np.array([3.0, 4.0]).reshape(1, 1, 1, 2)
+    y = oracle.output_gate(o, np.zeros_like(o), np.array([[1.0, 2.0]]), eps=0.0)
+    np.testing.assert_allclose(y.ravel(), [0.5 * 3.0 / math.sqrt(12.5), 0.5 * 2.0 * 4.0 / math.sqrt(12.5)], rtol=1e-15)
+    rs = np.random.default_rng(6)
+    o = rs.standard_normal((2, 3, 5, 16))
+    gate = rs.standard_normal((2, 3, 5, 16))
+    w = rs.standard_normal((3, 16))
+    y = oracle.output_gate(o, gate, w, eps=0.0)
+    # RMSNorm is invariant to a positive rescaling of the row
+    np.testing.assert_allclose(oracle.output_gate(7.5 * o, gate, w, eps=0.0), y, rtol=1e-13)
+    # with unit weights and an open gate (large logits) the rows have unit RMS
+    yy = oracle.output_gate(o, np.full_like(o, 60.0), np.ones((3, 16)), eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(yy * yy, axis=-1)), 1.0, rtol=1e-12)
+    # the weight is per head: head 1 only sees w[1]
+    w2 = w.copy()
+    w2[0] *= 3.0
+    np.testing.assert_allclose(oracle.output_gate(o, gate, w2, eps=0.0)[:, 1:], y[:, 1:], rtol=0, atol=0)
