@@ -248,6 +248,27 @@ kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_w
   return kda::launch_out_gate(a, (cudaStream_t)stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_kcp_compose(const float *M, const float *St, const float *h0, float *S_in, int R, int B,
+                             int H, int dk, int dv, kda_stream_t stream) {
+  if (R < 0 || B < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+  if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  const size_t n = (size_t)B * H;
+  if (n == 0) return KDA_OK;
+  if (!S_in || (R > 0 && (!M || !St))) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {R > 0 ? M : nullptr, R > 0 ? St : nullptr, h0, S_in};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+  const Range rs = range_of(S_in, n * dk * dv * 4), rm = range_of(M, R > 0 ? (size_t)R * n * dk * dk * 4 : 0),
+              rt = range_of(St, R > 0 ? (size_t)R * n * dk * dv * 4 : 0), rh = range_of(h0, h0 ? n * dk * dv * 4 : 0);
+  if (overlap(rs, rm) || overlap(rs, rt) || overlap(rs, rh)) return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  return kda::launch_kcp_compose(M, St, h0, S_in, R, (int)n, dk, dv, (cudaStream_t)stream) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
                                 const void *beta, float *S, void *o, int B, int H, int dk, int dv,
                                 kda_dtype_t dtype, float scale, kda_stream_t stream) {

@@ -50,6 +50,8 @@ struct OutGateArgs {
 };
 
 cudaError_t launch_out_gate(const OutGateArgs &a, cudaStream_t s);
+cudaError_t launch_kcp_compose(const float *M, const float *St, const float *h0, float *S_in, int R, int BH, int dk,
+                               int dv, cudaStream_t s);
 cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t s);
 // Planning of the tensor-core path: segments per chain, segment length, workspace bytes.

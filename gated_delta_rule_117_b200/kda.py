@@ -24,7 +24,8 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
                 "KDA_ERR_UNSUPPORTED", "KDA_ERR_DEVICE"]
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
-            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate"]
+            "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate",
+            "kda_kcp_compose"]
 
 
 class KdaError(RuntimeError):
@@ -65,6 +66,8 @@ def load_library():
             lib.kda_chunk_fwd_gated.restype = i
             lib.kda_output_gate.argtypes = [vp, vp, vp, f, vp] + [i] * 5 + [vp]
             lib.kda_output_gate.restype = i
+            lib.kda_kcp_compose.argtypes = [vp] * 4 + [i] * 5 + [vp]
+            lib.kda_kcp_compose.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
             lib.kda_recurrent_step.restype = i
             lib.kda_status_string.argtypes = [i]
@@ -130,6 +133,11 @@ def kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk,
 def kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream) -> int:
     """Eq. 6 output edge: y = Sigmoid(gate) * RMSNorm(o).  Returns the raw kda_status_t."""
     return load_library().kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream)
+
+
+def kda_kcp_compose(M, St, h0, S_in, R, B, H, dk, dv, stream) -> int:
+    """Cross-device KCP prefix: S_in from the gathered (M_r, S~_r) of the R earlier segments."""
+    return load_library().kda_kcp_compose(M, St, h0, S_in, R, B, H, dk, dv, stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:

@@ -205,6 +205,25 @@ kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_w
                              int B, int H, int T, int dv, kda_dtype_t dtype, kda_stream_t stream);
 
 /*
+ * Cross-device KDA context parallelism, prefix step (Kimi K3 report, section
+ * 5.1.2, Eq. 17).  Each rank holds one segment of every chain; a segment maps
+ * its entering state S to S~ + M S.  After one all-gather of the (M_r, S~_r)
+ * pairs (the caller's NCCL collective), rank R composes the state entering its
+ * segment,
+ *     S_in = M_{R-1} (... (M_0 h0 + S~_0) ...) + S~_{R-1},
+ * and runs its prefill from S_in.  (M_r, S~_r) of a segment come from two
+ * prefill calls on it: S~ = h_T from a zero state, M = h_T from h0 = I with
+ * v = 0 (dk == dv).
+ *   M    : [R, B, H, dk, dk] fp32;  St : [R, B, H, dk, dv] fp32 (rank-major)
+ *   h0   : [B, H, dk, dv] fp32, or NULL for a zero initial state
+ *   S_in : [B, H, dk, dv] fp32, written; must not overlap the inputs
+ *   R    : number of earlier segments (0 on the first rank: S_in = h0)
+ * All pointers 16-byte aligned; dk, dv one of 16, 32, 64, 128.
+ */
+kda_status_t kda_kcp_compose(const float *M, const float *St, const float *h0, float *S_in, int R, int B,
+                             int H, int dk, int dv, kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

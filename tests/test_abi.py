@@ -169,6 +169,18 @@ def test_output_gate_in_place_and_empty(lib):
         assert st in (7, 9)
 
 
+@pytest.mark.parametrize("over,code", [
+    (dict(R=-1), 1), (dict(S_in=None), 1), (dict(M=None), 1), (dict(dk=24), 2),
+    (dict(St=BASE + (1 << 20) + 4), 4),
+    (dict(S_in=BASE), 5),                 # S_in overlaps M
+])
+def test_kcp_compose_rejects(lib, over, code):
+    a = dict(M=BASE, St=BASE + (1 << 20), h0=BASE + (2 << 20), S_in=BASE + (3 << 20), R=2, B=1, H=2, dk=64, dv=64,
+             stream=None)
+    a.update(over)
+    assert kda.kda_kcp_compose(**a) == code
+
+
 def _dcall(**over):
     B, H, dk, dv = 4, 2, 16, 16
     n = 4096

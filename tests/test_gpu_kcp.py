@@ -1,0 +1,66 @@
+"""Cross-device KDA context parallelism (Kimi K3 report, section 5.1.2,
+Eq. 17) on one device: the per-segment transitions, the prefix composition
+(kda_kcp_compose) and the per-segment prefill, run for R emulated ranks in
+rank order, reproduce the oracle over the whole sequence.  (The exchange
+itself is an all-gather; its orchestration is tested on gloo ranks.)"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_117_b200 import kda, synth
+from gated_delta_rule_117_b200.kcp import LibkdaOps
+from parity_util import TOL, oracle_prefill, rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _emulate(d, R, T):
+    n = T // R
+    seg = lambda r: [d[k][:, :, r * n:(r + 1) * n].contiguous() for k in ("q", "k", "v", "g", "beta")]
+    pairs = [LibkdaOps.transition(*seg(r)) for r in range(R)]  # every rank's (S~, M)
+    outs, hT = [], None
+    for r in range(R):  # rank r after the all-gather
+        s_in = LibkdaOps.compose([m for _, m in pairs[:r]], [st for st, _ in pairs[:r]], d["h0"], d["h0"])
+        o, hT = LibkdaOps.prefill(*seg(r), s_in)
+        outs.append(o)
+    return torch.cat(outs, dim=2), hT
+
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_tensor_core_path(R):
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=4, T=960, seed=70 + R)
+    x = synth.prefill_inputs(w)
+    o, hT = _emulate(to_dev(x), R, w.T)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_cuda_core_path_fp32():
+    w = synth.WORKLOADS["tiny_f32"].with_(H=3, T=192, h0_std=0.05, seed=75)
+    x = synth.prefill_inputs(w)
+    o, hT = _emulate(to_dev(x), 4, w.T)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["f32"] and rel_l2(hT, h_ref) <= TOL["f32"]
+
+
+def test_compose_matches_fp64():
+    rs = np.random.default_rng(76)
+    R, B, H, dk, dv = 3, 2, 2, 64, 32
+    M = rs.standard_normal((R, B, H, dk, dk)) / np.sqrt(dk)
+    St = rs.standard_normal((R, B, H, dk, dv))
+    h0 = rs.standard_normal((B, H, dk, dv))
+    ref = h0.copy()
+    for r in range(R):
+        ref = M[r] @ ref + St[r]
+    # keep the device copies alive while the call uses their addresses
+    Md, Sd, hd = (torch.from_numpy(a).float().cuda() for a in (M, St, h0))
+    out = torch.empty(B, H, dk, dv, device="cuda")
+    st = kda.kda_kcp_compose(Md.data_ptr(), Sd.data_ptr(), hd.data_ptr(), out.data_ptr(), R, B, H, dk, dv, None)
+    assert st == 0
+    assert rel_l2(out, ref) <= 1e-5
+    # first rank: no earlier segment, the entering state is h0
+    assert kda.kda_kcp_compose(None, None, hd.data_ptr(), out.data_ptr(), 0, B, H, dk, dv, None) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out, hd)

@@ -53,3 +53,67 @@ def test_single_process_helpers():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.job_throughput(4096, 1, 2.0) == pytest.approx(4096 / 0.002)
+
+
+# ---- cross-device KCP orchestration (gloo, 2 ranks, CPU stand-ins) ----------
+
+class _OracleOps:
+    """The KCP steps on the CPU with the fp64 oracle (test stand-ins for the
+    device kernels): the orchestration, not the arithmetic, is under test."""
+
+    @staticmethod
+    def transition(q, k, v, g, beta, scale=0.0):
+        import numpy as np
+        import oracle
+        a = [t.double().numpy() for t in (q, k, v, g, beta)]
+        _, st = oracle.recurrent(*a)
+        dk = q.shape[-1]
+        eye = np.broadcast_to(np.eye(dk), q.shape[:2] + (dk, dk)).copy()
+        _, m = oracle.recurrent(a[0], a[1], np.zeros_like(a[2]), a[3], a[4], eye)
+        return torch.from_numpy(st), torch.from_numpy(m)
+
+    @staticmethod
+    def compose(ms, sts, h0, like):
+        s = torch.zeros_like(like, dtype=torch.float64) if h0 is None else h0.double().clone()
+        for m, st in zip(ms, sts):
+            s = m @ s + st
+        return s
+
+    @staticmethod
+    def prefill(q, k, v, g, beta, h0, scale=0.0):
+        import oracle
+        a = [t.double().numpy() for t in (q, k, v, g, beta)]
+        o, hT = oracle.recurrent(*a, h0.double().numpy())
+        return torch.from_numpy(o), torch.from_numpy(hT)
+
+
+def _kcp_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from gated_delta_rule_117_b200 import kcp, synth
+        w = synth.WORKLOADS["tiny_f32"].with_(H=2, T=90, h0_std=0.05, seed=21)
+        x = synth.prefill_inputs(w)
+        n = w.T // world
+        sl = {k2: (x[k2][:, :, rank * n:(rank + 1) * n] if k2 != "h0" else x[k2]) for k2 in x}
+        o, hT = kcp.kcp_prefill(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], x["h0"], ops=_OracleOps)
+        out[rank] = (o.numpy(), hT.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cross_device_kcp_orchestration_two_ranks():
+    import numpy as np
+    import oracle
+    from gated_delta_rule_117_b200 import synth
+    world, port = 2, _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_kcp_worker, args=(world, port, out), nprocs=world, join=True)
+    w = synth.WORKLOADS["tiny_f32"].with_(H=2, T=90, h0_std=0.05, seed=21)
+    x = synth.prefill_inputs(w)
+    o_ref, h_ref = oracle.recurrent(*[x[n].double().numpy() for n in ("q", "k", "v", "g", "beta", "h0")])
+    o = np.concatenate([out[0][0], out[1][0]], axis=2)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-12)        # rank r's tokens, in rank order
+    np.testing.assert_allclose(out[1][1], h_ref, rtol=1e-10, atol=1e-12)  # last rank: the final state
