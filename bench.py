@@ -298,13 +298,15 @@ def main():
         "gpu_launches": plan["launches"] * args.steps,
     }
     if world == 1 and T >= CKPT_INTERVAL:
-        result["ckpt"] = measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step)
+        result["ckpt"] = optional_leg(lambda: measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step))
     if world == 1:
-        result["out_gate"] = measure_out_gate(args, w, o, flush, kda, torch, pk)
+        result["out_gate"] = optional_leg(lambda: measure_out_gate(args, w, o, flush, kda, torch, pk))
     if world == 1 and B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
-        result["gate"] = measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, ms_per_step)
+        result["gate"] = optional_leg(lambda: measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch,
+                                                           ms_per_step))
     if not args.no_decode and world == 1:
         result["decode"] = measure_decode(args, synth, kda, torch, dev, pk, pk_kind)
+        result["spec"] = optional_leg(lambda: measure_spec(args, synth, kda, torch, dev, pk))
     clocks = clk.summary()
     result["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -318,6 +320,15 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result))
+
+
+def optional_leg(fn):
+    """A secondary measurement (checkpoints, fused gate, output edge, replay):
+    a failure there is recorded in its own object and never costs the main line."""
+    try:
+        return fn()
+    except Exception as ex:  # noqa: BLE001
+        return {"error": "%s: %s" % (type(ex).__name__, ex)}
 
 
 CKPT_INTERVAL = 512  # hash-block size of the prefix cache (tokens)
@@ -469,6 +480,48 @@ def measure_e2e(args, w, x, kda, torch, dev, plan):
     ms = a.elapsed_time(b) / args.steps
     return {"value": B * T / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms}
+
+
+SPEC_WINDOW, SPEC_REPLAY = 4, 2  # window of 4 tokens: 2 accepted drafts replayed, bonus + 1 draft verified
+
+
+def measure_spec(args, synth, kda, torch, dev, pk):
+    """Speculative-decode replay and verify on the decode workload's state
+    (B256 H32, 512 MiB fp32): one kda_spec_replay_verify per window of
+    SPEC_WINDOW tokens, SPEC_REPLAY of them replayed and committed.  The state
+    is read once and written once per window."""
+    w = synth.WORKLOADS["decode_b256_h32"]
+    x = synth.decode_inputs(w, steps=SPEC_WINDOW)
+    S = x["S0"].to(dev)
+    # window inputs [B, H, W, d] from the first SPEC_WINDOW pre-generated steps
+    win = {n: x[n][:SPEC_WINDOW].movedim(0, 2).contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
+    o = torch.empty(w.B, w.H, SPEC_WINDOW, w.dv, dtype=w.torch_dtype, device=dev)
+    nr = torch.full((w.B,), SPEC_REPLAY, dtype=torch.int32, device=dev)
+    sp = torch.cuda.current_stream().cuda_stream
+
+    def one():
+        st = kda.kda_spec_replay_verify(win["q"].data_ptr(), win["k"].data_ptr(), win["v"].data_ptr(),
+                                        win["g"].data_ptr(), win["beta"].data_ptr(), S.data_ptr(), o.data_ptr(),
+                                        nr.data_ptr(), w.B, w.H, SPEC_WINDOW, w.dk, w.dv, kda.KDA_DTYPE_BF16, 0.0, sp)
+        if st != 0:
+            raise kda.KdaError(st, "kda_spec_replay_verify")
+
+    for _ in range(max(args.warmup, 3)):
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(16)]
+    for a, b in ev:
+        a.record()
+        one()
+        b.record()
+    torch.cuda.synchronize()
+    med = statistics.median(a.elapsed_time(b) for a, b in ev)
+    e = 2
+    nbytes = (2 * S.numel() * 4 + w.B * w.H * SPEC_WINDOW * (3 * w.dk + w.dv + 1) * e
+              + w.B * w.H * (SPEC_WINDOW - SPEC_REPLAY) * w.dv * e)
+    gbs = nbytes / (med / 1e3) / 1e9
+    return {"window": SPEC_WINDOW, "replayed": SPEC_REPLAY, "ms_per_window_median": med, "bytes_per_window": nbytes,
+            "GB/s": gbs, "frac_of_hbm_peak": gbs / pk["hbm_gbs"], "gpu_launches": len(ev)}
 
 
 def measure_decode(args, synth, kda, torch, dev, pk, pk_kind):

@@ -269,6 +269,40 @@ kda_status_t kda_kcp_compose(const float *M, const float *St, const float *h0, f
              : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v, const void *g,
+                                    const void *beta, float *S, void *o, const int *n_replay, int B,
+                                    int H, int W, int dk, int dv, kda_dtype_t dtype, float scale,
+                                    kda_stream_t stream) {
+  if (B < 0 || H < 0 || W < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+  if (B * H == 0 || W == 0) return KDA_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o || !n_replay) return KDA_ERR_INVALID_ARG;
+  const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(S) || ((uintptr_t)n_replay & 3u) != 0) return KDA_ERR_ALIGNMENT;
+  const void *ptrs[] = {q, k, v, g, beta, o};
+  for (const void *p : ptrs)
+    if (((uintptr_t)p % e) != 0) return KDA_ERR_ALIGNMENT;
+  const size_t n = (size_t)B * H;
+  const Range rq = range_of(q, n * W * dk * e), rk = range_of(k, n * W * dk * e), rv = range_of(v, n * W * dv * e),
+              rg = range_of(g, n * W * dk * e), rb = range_of(beta, n * W * e), rn = range_of(n_replay, (size_t)B * 4),
+              rS = range_of(S, n * dk * dv * 4), ro = range_of(o, n * W * dv * e);
+  const Range ins[] = {rq, rk, rv, rg, rb, rn};
+  for (const Range &r : ins)
+    if (overlap(ro, r) || overlap(rS, r)) return KDA_ERR_ALIAS;
+  if (overlap(ro, rS)) return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  kda::SpecArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o; a.n_replay = n_replay;
+  a.B = B; a.H = H; a.W = W; a.dk = dk; a.dv = dv;
+  a.bf16 = dtype == KDA_DTYPE_BF16;
+  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
+  return kda::launch_spec_replay_verify(a, (cudaStream_t)stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
                                 const void *beta, float *S, void *o, int B, int H, int dk, int dv,
                                 kda_dtype_t dtype, float scale, kda_stream_t stream) {

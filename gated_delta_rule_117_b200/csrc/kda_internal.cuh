@@ -49,6 +49,17 @@ struct OutGateArgs {
   float eps;
 };
 
+struct SpecArgs {
+  const void *q, *k, *v, *g, *beta;
+  float *S;
+  void *o;
+  const int *n_replay;  // [B] accepted tokens to replay per sequence (device)
+  int B, H, W, dk, dv;
+  int bf16;
+  float scale;
+};
+
+cudaError_t launch_spec_replay_verify(const SpecArgs &a, cudaStream_t s);
 cudaError_t launch_out_gate(const OutGateArgs &a, cudaStream_t s);
 cudaError_t launch_kcp_compose(const float *M, const float *St, const float *h0, float *S_in, int R, int BH, int dk,
                                int dv, cudaStream_t s);

@@ -25,7 +25,7 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
             "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate",
-            "kda_kcp_compose"]
+            "kda_kcp_compose", "kda_spec_replay_verify"]
 
 
 class KdaError(RuntimeError):
@@ -68,6 +68,8 @@ def load_library():
             lib.kda_output_gate.restype = i
             lib.kda_kcp_compose.argtypes = [vp] * 4 + [i] * 5 + [vp]
             lib.kda_kcp_compose.restype = i
+            lib.kda_spec_replay_verify.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
+            lib.kda_spec_replay_verify.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
             lib.kda_recurrent_step.restype = i
             lib.kda_status_string.argtypes = [i]
@@ -138,6 +140,12 @@ def kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream) -> 
 def kda_kcp_compose(M, St, h0, S_in, R, B, H, dk, dv, stream) -> int:
     """Cross-device KCP prefix: S_in from the gathered (M_r, S~_r) of the R earlier segments."""
     return load_library().kda_kcp_compose(M, St, h0, S_in, R, B, H, dk, dv, stream)
+
+
+def kda_spec_replay_verify(q, k, v, g, beta, S, o, n_replay, B, H, W, dk, dv, dtype, scale, stream) -> int:
+    """Speculative-decode replay and verify over a W-token window.  Returns the raw kda_status_t."""
+    return load_library().kda_spec_replay_verify(q, k, v, g, beta, S, o, n_replay, B, H, W, dk, dv, dtype, scale,
+                                                 stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
@@ -263,6 +271,22 @@ def output_gate(o, gate, rms_weight, eps=1e-6, *, y=None, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_output_gate")
     return y
+
+
+def spec_replay_verify(q, k, v, g, beta, S, n_replay, *, o=None, scale=0.0, stream=None):
+    """Window of W tokens per sequence ([B, H, W, d]): replay the first
+    n_replay[b] (accepted, committed to S in place), verify the rest (o).
+    n_replay: [B] int32 CUDA tensor.  Returns o."""
+    import torch
+    B, H, W, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.zeros(B, H, W, dv, dtype=q.dtype, device=q.device)
+    st = kda_spec_replay_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), _ptr(n_replay),
+                                B, H, W, dk, dv, _dtype_code(q), float(scale), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_spec_replay_verify")
+    return o
 
 
 def recurrent_step(q, k, v, g, beta, S, *, o=None, scale=0.0, stream=None):

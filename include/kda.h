@@ -224,6 +224,30 @@ kda_status_t kda_kcp_compose(const float *M, const float *St, const float *h0, f
                              int H, int dk, int dv, kda_stream_t stream);
 
 /*
+ * Speculative-decode replay and verify (Kimi K3 report, section 5.4.2): one
+ * recurrent loop over a window of W tokens per sequence.  The first
+ * n_replay[b] tokens are the accepted drafts of the previous verification,
+ * whose projected inputs the caller cached: they advance the committed state,
+ * which is written back to S after the last of them.  The remaining tokens
+ * (bonus token and next draft) advance the state on chip only and write their
+ * outputs o for verification; S never sees them.
+ *
+ *   q, k, g  : [B, H, W, dk] dtype;  v : [B, H, W, dv] dtype;  beta : [B, H, W] dtype
+ *   S        : [B, H, dk, dv] fp32, 16-byte aligned, updated in place (unchanged
+ *              when n_replay[b] == 0)
+ *   o        : [B, H, W, dv] dtype; rows t >= n_replay[b] are written, the
+ *              others are left as they were
+ *   n_replay : [B] int32 in device memory; values are clamped to [0, W]
+ *   dk, dv   : each one of 16, 32, 64, 128;  scale as for kda_chunk_fwd.
+ * Element-aligned inputs; o must not overlap S or any input; S must not
+ * overlap any input.
+ */
+kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v, const void *g,
+                                    const void *beta, float *S, void *o, const int *n_replay, int B,
+                                    int H, int W, int dk, int dv, kda_dtype_t dtype, float scale,
+                                    kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

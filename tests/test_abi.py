@@ -181,6 +181,19 @@ def test_kcp_compose_rejects(lib, over, code):
     assert kda.kda_kcp_compose(**a) == code
 
 
+@pytest.mark.parametrize("over,code", [
+    (dict(W=-1), 1), (dict(n_replay=None), 1), (dict(dk=8), 2), (dict(dtype=3), 3),
+    (dict(S=BASE + (1 << 22) + 8), 4), (dict(n_replay=BASE + (3 << 22) + 2), 4),
+    (dict(o=BASE + (1 << 22)), 5),       # o inside S
+])
+def test_spec_replay_verify_rejects(lib, over, code):
+    a = dict(q=BASE, k=BASE + 65536, v=BASE + 2 * 65536, g=BASE + 3 * 65536, beta=BASE + 4 * 65536, S=BASE + (1 << 22),
+             o=BASE + (2 << 22), n_replay=BASE + (3 << 22), B=2, H=2, W=4, dk=64, dv=64, dtype=1, scale=0.0,
+             stream=None)
+    a.update(over)
+    assert kda.kda_spec_replay_verify(**a) == code
+
+
 def _dcall(**over):
     B, H, dk, dv = 4, 2, 16, 16
     n = 4096
