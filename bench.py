@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -67,7 +68,7 @@ class ClockSampler:
     def __init__(self, device_id: str):
         self.dev = device_id  # nvidia-smi -i accepts the GPU UUID (robust to CUDA_VISIBLE_DEVICES)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+        self.path = os.path.join(tempfile.gettempdir(), "kda_bench_clocks_%d.csv" % os.getpid())
 
     def __enter__(self):
         try:
