@@ -64,3 +64,82 @@ def test_mutant_is_caught(tmp_path, name):
     o_mut, h_mut = _run(lib, q, k, v, g, beta, h0, 0.6)
     # the real oracle passes the brute-force pin (test_oracle.py); the mutant must differ
     assert not (np.allclose(o_mut, o_ref, atol=1e-9) and np.allclose(h_mut, h_ref, atol=1e-9))
+
+
+# ---- planted mistakes in the fp64 restatements of Eq. 5 and Eq. 6 ----------
+
+def _gate_pins(gate):
+    """The checks test_oracle's gate pin makes, against a candidate gate(z, A, g_min)."""
+    A = np.array([[0.0, np.log(2.0)], [-1.0, 0.5]])
+    z = np.array([[[[1.0, 1.0]], [[-2.0, 3.0]]]])
+    ref = -5.0 / (1.0 + np.exp(-np.array([[[1.0, 2.0]], [[-2.0 * np.exp(-1.0), 3.0 * np.exp(0.5)]]])))
+    ok = np.allclose(gate(np.zeros((1, 2, 1, 2)), A, -5.0), -2.5, rtol=0, atol=1e-15)
+    ok &= np.allclose(gate(z, A, -5.0)[0], ref, rtol=1e-15)
+    zz = np.random.default_rng(5).standard_normal((2, 2, 50, 2)) * 3
+    gg = gate(zz, A, -5.0)
+    ok &= bool(np.all(gg > -5.0) and np.all(gg < 0.0))
+    ok &= np.allclose(gate(zz, A, -2.0), gg * 0.4, rtol=1e-14)
+    return bool(ok)
+
+
+GATE_MUTANTS = {
+    "no_scale": lambda z, A, gm: gm / (1.0 + np.exp(-np.asarray(z))),
+    "scale_not_exponentiated": lambda z, A, gm: gm / (1.0 + np.exp(-np.asarray(A)[:, None, :] * z)),
+    "wrong_sigmoid_side": lambda z, A, gm: gm / (1.0 + np.exp(np.exp(np.asarray(A))[:, None, :] * z)),
+    "scale_of_channel_0_only": lambda z, A, gm: gm / (1.0 + np.exp(-np.exp(np.asarray(A)[:, None, :1]) * z)),
+}
+
+
+def test_gate_pins_hold_for_the_oracle():
+    assert _gate_pins(oracle.gate)
+
+
+@pytest.mark.parametrize("name", sorted(GATE_MUTANTS))
+def test_gate_mutant_is_caught(name):
+    assert not _gate_pins(GATE_MUTANTS[name])
+
+
+def _output_gate_pins(fn):
+    o = np.array([3.0, 4.0]).reshape(1, 1, 1, 2)
+    y = fn(o, np.zeros_like(o), np.array([[1.0, 2.0]]), 0.0)
+    ok = np.allclose(y.ravel(), [0.5 * 3.0 / np.sqrt(12.5), 0.5 * 2.0 * 4.0 / np.sqrt(12.5)], rtol=1e-15)
+    rs = np.random.default_rng(6)
+    o = rs.standard_normal((2, 3, 5, 16))
+    gate = rs.standard_normal((2, 3, 5, 16))
+    w = rs.standard_normal((3, 16))
+    y = fn(o, gate, w, 0.0)
+    ok &= np.allclose(fn(7.5 * o, gate, w, 0.0), y, rtol=1e-13)
+    yy = fn(o, np.full_like(o, 60.0), np.ones((3, 16)), 0.0)
+    ok &= np.allclose(np.sqrt(np.mean(yy * yy, axis=-1)), 1.0, rtol=1e-12)
+    w2 = w.copy()
+    w2[0] *= 3.0
+    ok &= np.array_equal(fn(o, gate, w2, 0.0)[:, 1:], y[:, 1:])
+    return bool(ok)
+
+
+def _og(norm, gate_act, weight_index):
+    def fn(o, gate, w, eps):
+        o = np.asarray(o, dtype=np.float64)
+        wv = np.asarray(w, dtype=np.float64)
+        wv = wv[:, None, :] if weight_index == "head" else wv[None, :1, None, :].reshape(1, 1, 1, -1)
+        return gate_act(np.asarray(gate)) * wv * o / norm(o, eps)
+    return fn
+
+
+_sig = lambda x: 1.0 / (1.0 + np.exp(-x))
+OUT_GATE_MUTANTS = {
+    "l2_norm_not_rms": _og(lambda o, e: np.sqrt(np.sum(o * o, axis=-1, keepdims=True) + e), _sig, "head"),
+    "mean_abs_norm": _og(lambda o, e: np.mean(np.abs(o), axis=-1, keepdims=True) + e, _sig, "head"),
+    "gate_not_sigmoid": _og(lambda o, e: np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + e), np.tanh, "head"),
+    "weight_of_head_0_everywhere": _og(lambda o, e: np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + e), _sig,
+                                       "first"),
+}
+
+
+def test_output_gate_pins_hold_for_the_oracle():
+    assert _output_gate_pins(oracle.output_gate)
+
+
+@pytest.mark.parametrize("name", sorted(OUT_GATE_MUTANTS))
+def test_output_gate_mutant_is_caught(name):
+    assert not _output_gate_pins(OUT_GATE_MUTANTS[name])
