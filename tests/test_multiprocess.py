@@ -103,17 +103,18 @@ def _kcp_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_cross_device_kcp_orchestration_two_ranks():
+@pytest.mark.parametrize("world", [2, 3])
+def test_cross_device_kcp_orchestration(world):
     import numpy as np
     import oracle
     from gated_delta_rule_117_b200 import synth
-    world, port = 2, _free_port()
+    port = _free_port()
     mgr = mp.Manager()
     out = mgr.dict()
     mp.spawn(_kcp_worker, args=(world, port, out), nprocs=world, join=True)
     w = synth.WORKLOADS["tiny_f32"].with_(H=2, T=90, h0_std=0.05, seed=21)
     x = synth.prefill_inputs(w)
     o_ref, h_ref = oracle.recurrent(*[x[n].double().numpy() for n in ("q", "k", "v", "g", "beta", "h0")])
-    o = np.concatenate([out[0][0], out[1][0]], axis=2)
-    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-12)        # rank r's tokens, in rank order
-    np.testing.assert_allclose(out[1][1], h_ref, rtol=1e-10, atol=1e-12)  # last rank: the final state
+    o = np.concatenate([out[r][0] for r in range(world)], axis=2)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-12)               # rank r's tokens, in rank order
+    np.testing.assert_allclose(out[world - 1][1], h_ref, rtol=1e-10, atol=1e-12)  # last rank: the final state
