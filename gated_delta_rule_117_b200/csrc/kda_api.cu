@@ -5,10 +5,11 @@
 #include <stdint.h>
 #include <string.h>
 
-#include <atomic>
+#include <mutex>
 
 #include "kda.h"
 #include "kda_internal.cuh"
+#include "kda_tmap.cuh"
 
 namespace kda {
 
@@ -19,17 +20,35 @@ __device__ unsigned g_status_word;
 
 namespace {
 constexpr int kMaxDevices = 64;
-std::atomic<unsigned *> g_status_ptr[kMaxDevices];
+// Address of g_status_word per device, valid for the context it was looked up
+// in (a context re-created after cudaDeviceReset loads the module anew).
+struct StatusCache {
+  std::mutex mu;
+  unsigned long long ctx[kMaxDevices] = {};
+  unsigned *addr[kMaxDevices] = {};
+} g_status_cache;
 }  // namespace
 
 unsigned *device_status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  unsigned *p = g_status_ptr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  {
+    std::lock_guard<std::mutex> lk(g_status_cache.mu);
+    if (have_id && g_status_cache.addr[dev] && g_status_cache.ctx[dev] == id) return g_status_cache.addr[dev];
+  }
   void *addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return nullptr;
-  g_status_ptr[dev].store((unsigned *)addr, std::memory_order_release);
+  if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess || !addr) {
+    (void)cudaGetLastError();  // leave no pending error for the caller's next runtime call
+    return nullptr;
+  }
+  if (!have_id) have_id = current_context_id(&id);  // the lookup made the primary context current
+  if (have_id) {
+    std::lock_guard<std::mutex> lk(g_status_cache.mu);
+    g_status_cache.ctx[dev] = id;
+    g_status_cache.addr[dev] = (unsigned *)addr;
+  }
   return (unsigned *)addr;
 }
 
@@ -182,8 +201,11 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
   a.g_min = g_min;
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
-  const cudaError_t ce = plan.path == KDA_PATH_TC32 ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
-                                                    : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
+  // T == 0 is a pure state copy (h_T = h0, or zeros): the CUDA-core kernel does
+  // that with no token to load, while the tensor-core path would need tensor
+  // maps over empty (possibly null) tensors
+  const cudaError_t ce = (plan.path == KDA_PATH_TC32 && T > 0) ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
+                                                               : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
   return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -1,4 +1,5 @@
-// Host-side TMA tensor-map encoding.  The driver entry point is fetched
+// Host-side uses of the CUDA driver API: TMA tensor-map encoding and the
+// identity of the current context.  The driver entry points are fetched
 // through the runtime (cudaGetDriverEntryPoint), so libkda needs no link
 // against libcuda.
 #include <cudaTypedefs.h>
@@ -12,16 +13,33 @@ namespace kda {
 namespace {
 PFN_cuTensorMapEncodeTiled g_encode = nullptr;
 std::once_flag g_once;
+PFN_cuCtxGetCurrent g_ctx_current = nullptr;
+PFN_cuCtxGetId g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+template <typename F>
+F driver_entry(const char *name) {
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(fn);
+  return nullptr;
+}
 }  // namespace
 
-bool tmap_available() {
-  std::call_once(g_once, [] {
-    void *fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+bool current_context_id(unsigned long long *id) {
+  std::call_once(g_ctx_once, [] {
+    g_ctx_current = driver_entry<PFN_cuCtxGetCurrent>("cuCtxGetCurrent");
+    g_ctx_id = driver_entry<PFN_cuCtxGetId>("cuCtxGetId");
   });
+  if (!g_ctx_current || !g_ctx_id) return false;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return g_ctx_id(ctx, id) == CUDA_SUCCESS;
+}
+
+bool tmap_available() {
+  std::call_once(g_once, [] { g_encode = driver_entry<PFN_cuTensorMapEncodeTiled>("cuTensorMapEncodeTiled"); });
   return g_encode != nullptr;
 }
 

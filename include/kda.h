@@ -34,8 +34,9 @@
  *    returns KDA_ERR_CUDA.  Errors raised on the device (a bounded wait that
  *    gave up) are recorded in a device status word read by
  *    kda_get_device_status().
- *  - Thread-safe: no global mutable host state besides a per-device cache of
- *    the status-word address filled on first use.
+ *  - Thread-safe: no global mutable host state besides a per-context cache of
+ *    the status-word address filled on first use (a context re-created after
+ *    cudaDeviceReset looks it up again).
  *  - No C++ exception crosses this interface.
  */
 #ifndef LIBKDA_KDA_H_
@@ -260,11 +261,14 @@ kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v,
  * fixed device array inside libkda of kda_noalloc_scratch_bytes() bytes
  * (32 MiB), held on every GPU that loads the library until the process exits.
  * Returns KDA_ERR_WORKSPACE if the call would need more scratch than that.
- * The first call on a device (with that device current) looks up the array's
- * device address once (cudaGetSymbolAddress); make that first call before any
- * stream capture.  No call allocates or frees memory.  All calls share the
- * array and nothing in it needs to start at zero; calls that overlap on the
- * GPU (different streams or host threads) race on it, so serialise them.
+ * Set-up: the first call that needs scratch in a CUDA context (with its
+ * device current) looks up the array's device address (cudaGetSymbolAddress)
+ * and caches it for that context; make that first call before any stream
+ * capture.  A context re-created after cudaDeviceReset repeats the lookup on
+ * its first call.  Plans that need no scratch never touch the array.  No call
+ * allocates or frees memory.  All calls share the array and nothing in it
+ * needs to start at zero; calls that overlap on the GPU (different streams or
+ * host threads) race on it, so serialise them.
  */
 kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
                                    const void *beta, const float *h0, void *o, float *h_T, int B,

@@ -167,9 +167,13 @@ def test_long_workload_full_sampled_head():
     assert torch.isfinite(o).all() and torch.isfinite(hT).all()
 
 
-def test_zero_length_copies_state():
-    w = synth.WORKLOADS["tiny_f32"].with_(T=0, h0_std=0.02)
+@pytest.mark.parametrize("dtype,d", [("f32", 16), ("bf16", 128)])
+def test_zero_length_copies_state(dtype, d):
+    # bf16 with d = 128 is the tensor-core plan: T = 0 must still copy h0 to h_T
+    w = synth.WORKLOADS["tiny_f32"].with_(T=0, h0_std=0.02, dtype=dtype, dk=d, dv=d, B=2, H=3)
     x = synth.prefill_inputs(w)
+    if dtype == "bf16":
+        assert kda.kda_chunk_fwd_plan(2, 3, 0, d, d, kda.KDA_DTYPE_BF16, 0)["path"] == kda.KDA_PATH_TC32
     o, hT = _run(x)
     assert o.numel() == 0 and torch.equal(hT.cpu(), x["h0"])
     o, hT = _run(x, use_h0=False)
