@@ -1,17 +1,29 @@
 #!/usr/bin/env python
 """Throughput of libkda's KDA forward on B200.
 
-Default line: chunked prefill (kda_chunk_fwd) on the prefill workload
-(B=1, H=16, T=4096, dk=dv=128, bf16 inputs, fp32 state, h0 ~ N(0, 0.02)),
-reported as tokens/s with algorithmic TFLOP/s and the HBM roofline fraction of
-the prefill kernel.  The same line carries the decode step (kda_recurrent_step,
-B=256, H=32, 64 steps, state updated in place) as GB/s against the HBM peak.
+Default line: chunked prefill (kda_chunk_fwd) on the long-context workload
+(B=1, H=16, T=2^20, dk=dv=128, bf16 inputs, fp32 state, h0 = 0; in-device
+context parallelism over the 148 SMs), reported as tokens/s with algorithmic
+TFLOP/s and the HBM roofline fraction of the prefill step.  The same line
+carries:
+  * `configs`: the other prefill workloads (B1 H16 T4096 with h0, B8 H32 T8192
+    with fast-decay heads), each timed the same way with its own roofline and
+    an oracle check of sampled whole chains;
+  * `decode`: the decode step (kda_recurrent_step, B=256, H=32, 64 steps,
+    state updated in place) as GB/s against the HBM peak;
+  * `parity` and `cpu_baseline`: the fp64 oracle over whole sampled chains of
+    the main workload (run on host cores while the GPU legs run), compared
+    with the timed run's own output, and its throughput;
+  * `e2e`: the same metric through the C ABI from pinned host buffers;
+  * secondary legs (checkpoints, output gate, fused gate, replay).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl libkda|reference]
 
-Under torchrun each rank runs an independent replica of the workload (the
-(batch, head) chains are independent: no collective on the data path), time is
-the max over ranks, and value is the whole-job throughput.
+With --gpus N > 1 the script starts N ranks itself (torch.distributed.run)
+unless a launcher already set WORLD_SIZE, which must then equal N.  Each rank
+runs an independent replica of the workload (the (batch, head) chains are
+independent: no collective on the data path), time is the max over ranks, and
+value is the whole-job throughput.
 """
 from __future__ import annotations
 
@@ -169,63 +181,123 @@ def cpu_oracle_prefill(w, x, threads):
     return time.perf_counter() - t0
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill_h16_t4k")
-    ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
-    ap.add_argument("--chunk-size", type=int, default=0)
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
-    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (for profiling)")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        ap.error("--warmup must be >= 3")
+ORACLE_BLOCK = 1 << 16  # tokens per oracle call; the state is carried between calls
 
-    from gated_delta_rule_117_b200 import synth
-    w = synth.WORKLOADS[args.workload]
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    if args.impl == "reference":
-        return run_reference(args, w, rank, world)
-
+def _oracle_chain(job):
+    """CPU-baseline leg, in a spawned worker: the fp64 oracle over one whole
+    (b, h) chain of the host inputs, token block by token block with the state
+    carried, into shared-memory o_ref / h_ref.  Returns the compute seconds."""
     import torch
-    import torch.distributed as dist
-    from gated_delta_rule_117_b200 import kda
-    from gated_delta_rule_117_b200 import build as kbuild
+    import oracle
+    x, b, h, o_ref, h_ref, use_h0 = job
+    T = x["q"].shape[2]
+    S = x["h0"][b, h].double().numpy() if use_h0 else None
+    secs = 0.0
+    for s in range(0, T, ORACLE_BLOCK):
+        e = min(T, s + ORACLE_BLOCK)
+        f = lambda n: x[n][b, h, s:e].double().numpy()
+        args = (f("q"), f("k"), f("v"), f("g"), f("beta"))
+        t0 = time.perf_counter()
+        o, S = oracle.recurrent(*args, S, nthreads=1)
+        secs += time.perf_counter() - t0
+        o_ref[s:e] = torch.from_numpy(o)
+    if S is None:  # T == 0
+        S = x["h0"][b, h].double().numpy() if use_h0 else 0.0 * x["h0"][b, h].double().numpy()
+    h_ref.copy_(torch.from_numpy(S))
+    return secs
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    kbuild.build()
-    kda.load_library()
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-    pk, pk_kind = peaks()
 
-    if args.decode_only:
-        print(json.dumps(measure_decode(args, synth, kda, torch, dev, pk, pk_kind)))
-        return
-    assert not w.decode, "main line is a prefill workload"
-    w = rank_workload(w, rank)
-    x = synth.prefill_inputs(w)
-    d = {k: v.to(dev) for k, v in x.items()}
-    h0 = d["h0"] if w.h0_std > 0 else None
+class OracleLeg:
+    """The oracle on whole sampled chains of a workload's host inputs.  It is
+    the CPU baseline (the oracle as it stands, one core per chain, compute time
+    only) and, compared with the GPU output of the timed run, the parity check
+    of that run.  Started in spawned processes before the GPU work so the CPU
+    time overlaps it."""
+
+    def __init__(self, w, x, chains, workers):
+        import torch
+        self.w, self.chains = w, chains
+        self.o_ref = [torch.empty(w.T, w.dv, dtype=torch.float64).share_memory_() for _ in chains]
+        self.h_ref = [torch.empty(w.dk, w.dv, dtype=torch.float64).share_memory_() for _ in chains]
+        ctx = torch.multiprocessing.get_context("spawn")
+        self.pool = ctx.Pool(max(1, min(workers, len(chains))))
+        self.t0 = time.perf_counter()
+        self.res = [self.pool.apply_async(_oracle_chain, ((x, b, h, o, hr, w.h0_std > 0),))
+                    for (b, h), o, hr in zip(chains, self.o_ref, self.h_ref)]
+
+    def finish(self, o_gpu, h_gpu, seg_len):
+        """o_gpu [n, T, dv], h_gpu [n, dk, dv]: the timed run's output on the sampled chains (host)."""
+        import numpy as np
+        secs = [r.get() for r in self.res]
+        wall = time.perf_counter() - self.t0
+        self.pool.close()
+        self.pool.join()
+        eo, eh, seg_worst = [], [], 0.0
+        for i in range(len(self.chains)):
+            ref = self.o_ref[i].numpy()
+            got = o_gpu[i].double().numpy()
+            eo.append(rel_l2_np(got, ref))
+            eh.append(rel_l2_np(h_gpu[i].double().numpy(), self.h_ref[i].numpy()))
+            for s in range(0, self.w.T, seg_len):
+                seg_worst = max(seg_worst, rel_l2_np(got[s:s + seg_len], ref[s:s + seg_len]))
+        tol = 3e-3 if self.w.dtype == "bf16" else 1e-5
+        parity = {"chains": [list(c) for c in self.chains], "o_rel_l2": eo, "hT_rel_l2": eh,
+                  "o_rel_l2_worst_segment": seg_worst, "segment_tokens": seg_len, "tol": tol,
+                  "pass": bool(max(eo + eh + [seg_worst]) <= tol),
+                  "reference": "fp64 C token recurrence (oracle) over each whole chain"}
+        n = len(self.chains)
+        cpu = {"value": n * self.w.T / max(secs) / self.w.H, "unit": "tokens/s", "cores": n, "kind": "oracle",
+               "sample": "%d whole chains (b, h) = %s of %d tokens, one core each, compute time of the slowest; "
+                         "tokens/s of the workload = chain-tokens/s / H; ran while the GPU legs ran (wall %.1f s)"
+                         % (n, [list(c) for c in self.chains], self.w.T, wall)}
+        return parity, cpu
+
+
+def rel_l2_np(x, ref):
+    import numpy as np
+    den = float(np.linalg.norm(ref))
+    return float(np.linalg.norm(x - ref) / (den if den > 0 else 1.0))
+
+
+def sample_chains(w):
+    """Chains whose whole output the oracle recomputes: first, last and a middle
+    one; in a workload with fast-decay heads, those heads as well."""
+    from gated_delta_rule_117_b200 import synth
+    c = [(0, 0), (w.B - 1, w.H - 1)]
+    if w.B * w.H > 2:
+        c.insert(1, (w.B // 2, w.H // 3))
+    for h in synth.fast_decay_heads(w).tolist()[:2]:
+        c.append((min(1, w.B - 1), h))
+    out = []
+    for x in c:
+        if x not in out:
+            out.append(x)
+    return out
+
+
+def host_inputs(synth, w, world):
+    """Seeded host inputs of a prefill workload; large ones are generated by a
+    pool of spawned processes into shared memory (same values bit for bit)."""
+    if w.B * w.H * w.T <= (1 << 20):
+        return synth.prefill_inputs(w)
+    workers = max(1, min(16, (os.cpu_count() or 1) // max(1, world)))
+    return synth.prefill_inputs_parallel(w, workers=workers)
+
+
+def time_prefill(args, w, d, plan, kda, torch, flush, dev, clk=None, dist=None):
+    """CUDA-event time of each of args.steps kda_chunk_fwd calls on device-resident
+    inputs, L2 flushed (outside the events) before each; W untimed warm-ups.
+    Returns (per-step ms, o, h_T)."""
     B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
     dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
-    plan = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)
+    h0 = d["h0"] if w.h0_std > 0 else None
     o = torch.empty(B, H, T, dv, dtype=w.torch_dtype, device=dev)
     hT = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     ws = torch.empty(max(plan["workspace"], 16), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    ptr = lambda t: None if t is None else t.data_ptr()
+    stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
+    ptr = lambda t: None if t is None else t.data_ptr()
 
     def step():
         st = kda.kda_chunk_fwd(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["g"]), ptr(d["beta"]), ptr(h0),
@@ -239,46 +311,181 @@ def main():
         step()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
+    if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+    if clk is not None:
         clk.soak(lambda: (flush.zero_(), step()), torch)
-        if world > 1:
+        if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()  # L2 flush between timed iterations (outside the events)
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-    times_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(times_ms), dist if world > 1 else None, dev)
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(B * T, world, ms_per_step)
-    kern_ms = statistics.mean(times_ms)  # one launch per step: the step is the kernel
-    bytes_per_launch = synth.prefill_bytes(w)
-    achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9
-    flops = synth.flops_per_token_head(dk, dv, 64) * B * H * T
-    tflops = flops / (kern_ms / 1e3) / 1e12
-    kernel_name = "chunk16_kernel" if plan["path"] == kda.KDA_PATH_SIMT16 else "chunk_tc_kernel"
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between timed iterations (outside the events)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev], o, hT
+
+
+def prefill_figures(w, plan, ms, pk, pk_kind, synth):
+    """Throughput, algorithmic TFLOP/s and the HBM roofline of one prefill step."""
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+    nbytes = synth.prefill_bytes(w)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    flop_tok = synth.flops_per_token_head(dk, dv, 64)
+    tflops = flop_tok * B * H * T / (ms / 1e3) / 1e12
+    kernel = "chunk16_kernel" if plan["path"] == 1 else "chunk_tc_kernel"
     # With in-device context parallelism one step is three launches (segment
     # transitions, the prefix scan, the final pass); the roofline then uses the
     # whole step's time, which is the conservative reading.
-    roofline_scope = "kernel" if plan["launches"] == 1 else "step (%d launches)" % plan["launches"]
-    src = (["gated_delta_rule_117_b200/csrc/kda_chunk_simt.cu"] if plan["path"] == kda.KDA_PATH_SIMT16
+    scope = "kernel" if plan["launches"] == 1 else "step (%d launches)" % plan["launches"]
+    src = (["gated_delta_rule_117_b200/csrc/kda_chunk_simt.cu"] if plan["path"] == 1
            else ["gated_delta_rule_117_b200/csrc/kda_chunk_tc.cu"])
-    trec = traffic_record("%s:%s" % (kernel_name, w.name), src)
+    trec = traffic_record("%s:%s" % (kernel, w.name), src)
     traffic = None
     if trec:
         # a segmented step records the DRAM bytes of all its launches, like `achieved`
         traffic = trec.get("dram_bytes_per_step", trec.get("dram_bytes_per_launch"))
+    return {
+        "tokens_per_s": B * T / (ms / 1e3),
+        "tflops": {"value": tflops, "flop_per_token_head": flop_tok, "frac_of_bf16_peak": tflops / pk["bf16_tflops"],
+                   "peak_kind": pk_kind},
+        "roofline": {"kernel": kernel, "scope": scope, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": nbytes, "peak_kind": pk_kind, "kernel_ms": ms},
+    }
 
-    e2e = measure_e2e(args, w, x, kda, torch, dev, plan)
+
+def measure_subconfig(args, name, synth, kda, torch, dev, flush, pk, pk_kind, world):
+    """Another prefill workload, timed like the main line, with the oracle on
+    sampled whole chains (in process: these chains are short)."""
+    import oracle
+    w = synth.WORKLOADS[name]
+    x = host_inputs(synth, w, world)
+    d = {k: v.to(dev) for k, v in x.items()}
+    dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
+    plan = kda.kda_chunk_fwd_plan(w.B, w.H, w.T, w.dk, w.dv, dt, args.chunk_size)
+    times, o, hT = time_prefill(args, w, d, plan, kda, torch, flush, dev)
+    ms = statistics.mean(times)
+    res = {"workload": name, "B": w.B, "H": w.H, "T": w.T, "segments": plan["segments"],
+           "launches_per_step": plan["launches"], "ms_per_step": ms, "steps": args.steps}
+    res.update(prefill_figures(w, plan, ms, pk, pk_kind, synth))
+    chains = sample_chains(w)
+    f = lambda t: t.double().numpy()
+    eo, eh = [], []
+    for b, h in chains:
+        o_ref, h_ref = oracle.recurrent(f(x["q"][b, h]), f(x["k"][b, h]), f(x["v"][b, h]), f(x["g"][b, h]),
+                                        f(x["beta"][b, h]), f(x["h0"][b, h]) if w.h0_std > 0 else None)
+        eo.append(rel_l2_np(f(o[b, h].cpu()), o_ref))
+        eh.append(rel_l2_np(f(hT[b, h].cpu()), h_ref))
+    res["parity"] = {"chains": [list(c) for c in chains], "o_rel_l2": eo, "hT_rel_l2": eh, "tol": 3e-3,
+                     "pass": bool(max(eo + eh) <= 3e-3)}
+    del d, o, hT
+    return res
+
+
+def relaunch_under_torchrun(n):
+    """`--gpus N` without a launcher: start N ranks of this same command."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+SUBCONFIGS = ("prefill_h16_t4k", "batched_b8_h32_t8k")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_h16_t1m")
+    ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
+    ap.add_argument("--chunk-size", type=int, default=0)
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the workload's T (smaller slices for profiling; 0 = the workload's own)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle leg (baseline and parity)")
+    ap.add_argument("--no-subconfigs", action="store_true", help="skip the other prefill workloads")
+    ap.add_argument("--no-legs", action="store_true", help="skip the secondary legs (ckpt, gates, replay)")
+    ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (for profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args.gpus))
+
+    from gated_delta_rule_117_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.seq_len > 0:
+        w = w.with_(T=args.seq_len, name="%s_T%d" % (w.name, args.seq_len))
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_117_b200 import kda
+    from gated_delta_rule_117_b200 import build as kbuild
+
+    assert not w.decode, "main line is a prefill workload"
+    w = rank_workload(w, rank)
+    # host inputs and the oracle processes come before the first CUDA call
+    x = host_inputs(synth, w, world)
+    leg = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        chains = sample_chains(w) if w.T < (1 << 18) else [(0, 5), (w.B - 1, w.H - 1)]
+        leg = OracleLeg(w, x, chains, workers=len(chains))
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    kbuild.build()
+    kda.load_library()
+    dev = torch.device("cuda", local)
+    pk, pk_kind = peaks()
+
+    if args.decode_only:
+        print(json.dumps(measure_decode(args, synth, kda, torch, dev, pk, pk_kind)))
+        return
+    d = {k: v.to(dev) for k, v in x.items()}
+    h0 = d["h0"] if w.h0_std > 0 else None
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+    dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
+    plan = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+        times_ms, o, hT = time_prefill(args, w, d, plan, kda, torch, flush, dev, clk=clk,
+                                       dist=dist if world > 1 else None)
+    total_ms = max_over_ranks(sum(times_ms), dist if world > 1 else None, dev)
+    ms_per_step = total_ms / args.steps
+    value = job_throughput(B * T, world, ms_per_step)
+    kern_ms = statistics.mean(times_ms)
+    fig = prefill_figures(w, plan, kern_ms, pk, pk_kind, synth)
+    # the timed run's own output on the chains the oracle recomputes
+    if leg is not None:
+        o_s = torch.stack([o[b, h] for b, h in leg.chains]).cpu()
+        h_s = torch.stack([hT[b, h] for b, h in leg.chains]).cpu()
+
+    e2e = measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=dist if world > 1 else None)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -286,36 +493,38 @@ def main():
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; report's KDA input distributions)",
         "config": {"workload": w.name, "B": B, "H": H, "T": T, "dk": dk, "dv": dv,
                    "chunk_size": plan["chunk_size"], "path": plan["path"], "segments": plan["segments"],
-                   "h0": "N(0,0.02)" if w.h0_std > 0 else "zeros", "l2": "flushed (256 MB write) between steps",
+                   "h0": "N(0,0.02)" if w.h0_std > 0 else "zeros",
+                   "l2": "flushed (256 MB write) between steps; inputs %.1f GB" % (synth.prefill_bytes(w) / 1e9),
                    "parallelism": "replicas" if world > 1 else "single"},
-        "tflops": {"value": tflops, "flop_per_token_head": synth.flops_per_token_head(dk, dv, 64),
-                   "frac_of_bf16_peak": tflops / pk["bf16_tflops"], "peak_kind": pk_kind},
-        "roofline": {"kernel": kernel_name, "scope": roofline_scope, "bound": "hbm", "achieved": achieved,
-                     "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": bytes_per_launch, "peak_kind": pk_kind,
-                     "kernel_ms": kern_ms},
+        "tflops": fig["tflops"],
+        "roofline": fig["roofline"],
         "e2e": e2e,
         "gpu_launches": plan["launches"] * args.steps,
     }
-    if world == 1 and T >= CKPT_INTERVAL:
-        result["ckpt"] = optional_leg(lambda: measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, ms_per_step))
-    if world == 1:
+    if world == 1 and not args.no_legs:
+        ws = torch.empty(max(plan["workspace"], 16), dtype=torch.uint8, device=dev)
+        if T >= CKPT_INTERVAL:
+            result["ckpt"] = optional_leg(lambda: measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch,
+                                                               kern_ms))
         result["out_gate"] = optional_leg(lambda: measure_out_gate(args, w, o, flush, kda, torch, pk))
-    if world == 1 and B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
-        result["gate"] = optional_leg(lambda: measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch,
-                                                           ms_per_step))
+        if B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
+            result["gate"] = optional_leg(lambda: measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch,
+                                                               kern_ms))
+        del ws
+    del d, o, hT
+    if world == 1 and not args.no_subconfigs:
+        result["configs"] = [optional_leg(lambda n=n: measure_subconfig(args, n, synth, kda, torch, dev, flush, pk,
+                                                                        pk_kind, world))
+                             for n in SUBCONFIGS if n != w.name]
     if not args.no_decode and world == 1:
         result["decode"] = measure_decode(args, synth, kda, torch, dev, pk, pk_kind)
-        result["spec"] = optional_leg(lambda: measure_spec(args, synth, kda, torch, dev, pk))
-    clocks = clk.summary()
-    result["clocks"] = clocks
-    if rank == 0 and world == 1 and not args.no_cpu:
-        threads = min(os.cpu_count() or 1, B * H)
-        secs = cpu_oracle_prefill(w, x, threads)
-        result["cpu_baseline"] = {"value": B * T / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                  "sample": "whole workload (%d chains x %d tokens), fp64 C recurrence, 1 pass"
-                                            % (B * H, T)}
+        if not args.no_legs:
+            result["spec"] = optional_leg(lambda: measure_spec(args, synth, kda, torch, dev, pk))
+    result["clocks"] = clk.summary()
+    if leg is not None:
+        parity, cpu = leg.finish(o_s, h_s, max(plan["segment_tokens"], 1))
+        result["parity"] = parity
+        result["cpu_baseline"] = cpu
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -439,29 +648,44 @@ def measure_out_gate(args, w, o, flush, kda, torch, pk):
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac_of_hbm_peak": gbs / pk["hbm_gbs"], "gpu_launches": len(ev)}
 
 
-def measure_e2e(args, w, x, kda, torch, dev, plan):
+def pin_host(torch, t):
+    """Page-lock a host tensor in place (cudaHostRegister) so copies from it
+    are true async DMA; returns (tensor, registered).  Falls back to a pinned
+    copy when registration is refused."""
+    nbytes = t.numel() * t.element_size()
+    if nbytes and t.is_contiguous():
+        try:
+            if int(torch.cuda.cudart().cudaHostRegister(t.data_ptr(), nbytes, 0)) == 0:
+                return t, True
+        except Exception:  # noqa: BLE001
+            pass
+    return t.pin_memory(), False
+
+
+def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
     """Same metric through the C ABI from pinned host buffers: each step copies
-    the inputs host->device, runs kda_chunk_fwd and copies o and h_T back."""
+    the inputs host->device (into the device buffers the timed run used), runs
+    kda_chunk_fwd and copies o and h_T back to pinned host memory."""
     stream = torch.cuda.current_stream()
-    hx = {k: v.pin_memory() for k, v in x.items()}
-    dx = {k: torch.empty_like(v, device=dev) for k, v in x.items()}
     B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
     use_h0 = w.h0_std > 0
+    names = ["q", "k", "v", "g", "beta"] + (["h0"] if use_h0 else [])
+    pinned = {n: pin_host(torch, x[n]) for n in names}
+    hx = {n: p[0] for n, p in pinned.items()}
     ho = torch.empty(B, H, T, dv, dtype=w.torch_dtype).pin_memory()
     hh = torch.empty(B, H, dk, dv, dtype=torch.float32).pin_memory()
     do = torch.empty(B, H, T, dv, dtype=w.torch_dtype, device=dev)
     dh = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     ws = torch.empty(max(plan["workspace"], 16), dtype=torch.uint8, device=dev)
     dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
-    names = ["q", "k", "v", "g", "beta"] + (["h0"] if use_h0 else [])
     h2d = sum(hx[n].numel() * hx[n].element_size() for n in names)
     d2h = ho.numel() * ho.element_size() + hh.numel() * hh.element_size()
 
     def step():
         for n in names:
-            dx[n].copy_(hx[n], non_blocking=True)
-        st = kda.kda_chunk_fwd(dx["q"].data_ptr(), dx["k"].data_ptr(), dx["v"].data_ptr(), dx["g"].data_ptr(),
-                               dx["beta"].data_ptr(), dx["h0"].data_ptr() if use_h0 else None, do.data_ptr(),
+            d[n].copy_(hx[n], non_blocking=True)
+        st = kda.kda_chunk_fwd(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["g"].data_ptr(),
+                               d["beta"].data_ptr(), d["h0"].data_ptr() if use_h0 else None, do.data_ptr(),
                                dh.data_ptr(), B, H, T, dk, dv, dt, args.chunk_size, 0.0, ws.data_ptr(), ws.numel(),
                                stream.cuda_stream)
         if st != 0:
@@ -469,18 +693,27 @@ def measure_e2e(args, w, x, kda, torch, dev, plan):
         ho.copy_(do, non_blocking=True)
         hh.copy_(dh, non_blocking=True)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.steps):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / args.steps
-    return {"value": B * T / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": ms}
+    try:
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist, dev)
+    finally:
+        for n, (t, reg) in pinned.items():
+            if reg:
+                torch.cuda.cudart().cudaHostUnregister(t.data_ptr())
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": job_throughput(B * T, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "warmup": 3,
+            "host_buffers": "pinned (page-locked in place where possible)"}
 
 
 SPEC_WINDOW, SPEC_REPLAY = 4, 2  # window of 4 tokens: 2 accepted drafts replayed, bonus + 1 draft verified

@@ -93,7 +93,10 @@ kda_status_t plan_prefill(int B, int H, int T, int dk, int dv, kda_dtype_t dtype
   const bool tc = chunk_size == 32 || (chunk_size == 0 && tc_ok);
   p.path = tc ? KDA_PATH_TC32 : KDA_PATH_SIMT16;
   p.chunk_size = tc ? 32 : 16;
-  p.segments = tc ? kda::tc32_segments(B * H, T) : 1;
+  int seg_len = T;
+  p.segments = 1;
+  if (tc) kda::tc32_plan(B * H, T, &p.segments, &seg_len);
+  p.segment_tokens = p.segments > 1 ? seg_len : T;
   p.launches = (B * H == 0) ? 0 : (p.segments > 1 ? 3 : 1);
   p.workspace = tc ? kda::tc32_workspace(B * H, T) : 0;
   *plan = p;

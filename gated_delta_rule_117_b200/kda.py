@@ -36,7 +36,7 @@ class KdaError(RuntimeError):
 
 class kda_plan_t(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("chunk_size", ctypes.c_int), ("segments", ctypes.c_int),
-                ("launches", ctypes.c_int), ("workspace", ctypes.c_size_t)]
+                ("launches", ctypes.c_int), ("workspace", ctypes.c_size_t), ("segment_tokens", ctypes.c_int)]
 
 
 _lib = None
@@ -102,7 +102,7 @@ def kda_chunk_fwd_plan(B, H, T, dk, dv, dtype, chunk_size=0):
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_plan")
     return dict(path=p.path, chunk_size=p.chunk_size, segments=p.segments, launches=p.launches,
-                workspace=p.workspace)
+                workspace=p.workspace, segment_tokens=p.segment_tokens)
 
 
 def kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dtype, chunk_size=0) -> int:

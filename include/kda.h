@@ -84,6 +84,7 @@ typedef struct {
   int segments;     /* in-device context-parallel segments per chain (1 = none) */
   int launches;     /* kernel launches per call */
   size_t workspace; /* bytes of workspace the call needs */
+  int segment_tokens; /* tokens per context-parallel segment (the last may be shorter); T if unsegmented */
 } kda_plan_t;
 
 /*
