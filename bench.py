@@ -507,6 +507,9 @@ def main():
             result["ckpt"] = optional_leg(lambda: measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch,
                                                                kern_ms))
         result["out_gate"] = optional_leg(lambda: measure_out_gate(args, w, o, flush, kda, torch, pk))
+        sep = result["out_gate"].get("ms") if isinstance(result.get("out_gate"), dict) else None
+        result["out_gate_fused"] = optional_leg(lambda: measure_outgate_fused(args, w, d, h0, hT, ws, flush, kda, torch,
+                                                                              kern_ms, sep))
         if B * H * T <= (1 << 17):  # z is regenerated on the host: small workloads only
             result["gate"] = optional_leg(lambda: measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch,
                                                                kern_ms))
@@ -613,6 +616,49 @@ def measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, plain_ms):
     e = 2 if w.dtype == "bf16" else 4
     return {"ms_per_step": ms, "overhead": ms / plain_ms - 1.0,
             "separate_gate_bytes_per_step": 2 * B * H * T * dk * e, "gpu_launches": len(ev) * launches}
+
+
+def measure_outgate_fused(args, w, d, h0, hT, ws, flush, kda, torch, plain_ms, sep_ms):
+    """The same step through kda_chunk_fwd_outgate (Eq. 6 output edge fused into
+    the output epilogue: y written instead of o, o never in memory) against the
+    plain step followed by the separate edge pass."""
+    B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
+    dev, sp = hT.device, torch.cuda.current_stream().cuda_stream
+    gen = torch.Generator(device=dev).manual_seed(7)
+    gate = torch.randn(B, H, T, dv, generator=gen, device=dev).to(w.torch_dtype)
+    wt = torch.ones(H, dv, dtype=torch.float32, device=dev)
+    y = torch.empty(B, H, T, dv, dtype=w.torch_dtype, device=dev)
+    dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
+    ptr = lambda t: None if t is None else t.data_ptr()
+
+    def step():
+        st = kda.kda_chunk_fwd_outgate(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["g"]), ptr(d["beta"]), ptr(h0),
+                                       gate.data_ptr(), wt.data_ptr(), 1e-6, y.data_ptr(), ptr(hT), B, H, T, dk, dv, dt,
+                                       args.chunk_size, 0.0, ws.data_ptr(), ws.numel(), sp)
+        if st != 0:
+            raise kda.KdaError(st, "kda_chunk_fwd_outgate")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    e = 2 if w.dtype == "bf16" else 4
+    launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
+    out = {"ms_per_step": ms, "vs_plain_step": ms / plain_ms - 1.0,
+           "round_trip_bytes_removed": 2 * B * H * T * dv * e, "gpu_launches": len(ev) * launches}
+    if sep_ms is not None:
+        out["unfused_ms_per_step"] = plain_ms + sep_ms
+        out["speedup_vs_unfused"] = (plain_ms + sep_ms) / ms
+    del gate, wt, y
+    return out
 
 
 def measure_out_gate(args, w, o, flush, kda, torch, pk):

@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kda.h"
@@ -51,6 +52,16 @@ unsigned *device_status_ptr() {
   }
   return (unsigned *)addr;
 }
+
+namespace {
+// Failure-detection test settings; production calls never change them.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s: far beyond any real wait
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_stall{0};
+}  // namespace
+
+uint64_t debug_wait_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+int debug_stall() { return g_stall.load(std::memory_order_relaxed); }
 
 }  // namespace kda
 
@@ -143,12 +154,27 @@ size_t kda_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, kda_dty
 
 namespace {
 
-// kda_chunk_fwd and kda_chunk_fwd_ckpt (ckpt == nullptr: no checkpoints).
-// g holds the logits z when A_log is set (fused Eq. 5 gate).
+// Optional parts of a prefill call: state checkpoints, the fused Eq. 5 gate
+// (g then holds the logits z), the fused Eq. 6 output edge (o then receives y).
+struct Extras {
+  float *ckpt = nullptr;
+  int ckpt_interval = 0;
+  const float *A_log = nullptr;
+  float g_min = 0.f;
+  const void *gate = nullptr;
+  const float *rms_w = nullptr;
+  float eps = 0.f;
+};
+
+// kda_chunk_fwd and its variants.
 kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
-                       const float *h0, void *o, float *h_T, float *ckpt, int ckpt_interval, const float *A_log,
-                       float g_min, int B, int H, int T, int dk, int dv, kda_dtype_t dtype, int chunk_size,
-                       float scale, void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+                       const float *h0, void *o, float *h_T, const Extras &x, int B, int H, int T, int dk, int dv,
+                       kda_dtype_t dtype, int chunk_size, float scale, void *workspace, size_t workspace_bytes,
+                       kda_stream_t stream) {
+  float *const ckpt = x.ckpt;
+  const int ckpt_interval = x.ckpt_interval;
+  const float *const A_log = x.A_log;
+  const float g_min = x.g_min;
   kda_plan_t plan;
   kda_status_t st = plan_prefill(B, H, T, dk, dv, dtype, chunk_size, &plan);
   if (st != KDA_OK) return st;
@@ -185,6 +211,13 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
   if (overlap(rc, ro) || overlap(rc, rhT) || overlap(rc, rw)) return KDA_ERR_ALIAS;
   const Range ra = range_of(A_log, A_log ? (size_t)H * dk * 4 : 0);
   if (overlap(ra, ro) || overlap(ra, rhT) || overlap(ra, rw) || overlap(ra, rc)) return KDA_ERR_ALIAS;
+  if (x.gate) {  // the output edge's inputs are read while y (in o) is written
+    if (!aligned16(x.gate) || !aligned16(x.rms_w)) return KDA_ERR_ALIGNMENT;
+    const Range rg2 = range_of(x.gate, n * T * dv * e), rw2 = range_of(x.rms_w, (size_t)H * dv * 4);
+    if (overlap(rg2, ro) || overlap(rw2, ro) || overlap(rg2, rhT) || overlap(rw2, rhT) || overlap(rg2, rw) ||
+        overlap(rw2, rw))
+      return KDA_ERR_ALIAS;
+  }
 
   st = check_device();
   if (st != KDA_OK) return st;
@@ -202,13 +235,29 @@ kda_status_t chunk_fwd(const void *q, const void *k, const void *v, const void *
   a.n_ckpt = n_ckpt;
   a.A_log = A_log;
   a.g_min = g_min;
+  a.wait_ns = kda::debug_wait_ns();
+  a.stall = kda::debug_stall();
+  a.gate = x.gate;
+  a.rms_w = x.rms_w;
+  a.eps = x.eps;
   if (!a.status) return KDA_ERR_CUDA;
   if (T == 0 && !h_T) return KDA_OK;
   // T == 0 is a pure state copy (h_T = h0, or zeros): the CUDA-core kernel does
   // that with no token to load, while the tensor-core path would need tensor
   // maps over empty (possibly null) tensors
-  const cudaError_t ce = (plan.path == KDA_PATH_TC32 && T > 0) ? kda::launch_chunk_tc32(a, (cudaStream_t)stream)
-                                                               : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
+  const bool tc = plan.path == KDA_PATH_TC32 && T > 0;
+  // the CUDA-core kernel has no fused output edge: it writes o into y's buffer
+  // and the edge kernel then turns it into y in place
+  if (!tc) a.gate = nullptr;
+  cudaError_t ce = tc ? kda::launch_chunk_tc32(a, (cudaStream_t)stream) : kda::launch_chunk_simt16(a, (cudaStream_t)stream);
+  if (ce == cudaSuccess && !tc && x.gate && T > 0) {
+    kda::OutGateArgs og;
+    og.o = o; og.gate = x.gate; og.w = x.rms_w; og.y = o;
+    og.B = B; og.H = H; og.T = T; og.dv = dv;
+    og.bf16 = dtype == KDA_DTYPE_BF16;
+    og.eps = x.eps;
+    ce = kda::launch_out_gate(og, (cudaStream_t)stream);
+  }
   return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -220,8 +269,8 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const vo
                            const void *beta, const float *h0, void *o, float *h_T, int B, int H,
                            int T, int dk, int dv, kda_dtype_t dtype, int chunk_size, float scale,
                            void *workspace, size_t workspace_bytes, kda_stream_t stream) {
-  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, nullptr, 0, nullptr, 0.f, B, H, T, dk, dv, dtype, chunk_size, scale,
-                   workspace, workspace_bytes, stream);
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, Extras(), B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
+                   workspace_bytes, stream);
 }
 
 kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, const void *g,
@@ -230,8 +279,11 @@ kda_status_t kda_chunk_fwd_ckpt(const void *q, const void *k, const void *v, con
                                 kda_dtype_t dtype, int chunk_size, float scale, void *workspace,
                                 size_t workspace_bytes, kda_stream_t stream) {
   if (ckpt_interval <= 0 || ckpt_interval % 64 != 0) return KDA_ERR_INVALID_ARG;
-  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, ckpt, ckpt_interval, nullptr, 0.f, B, H, T, dk, dv, dtype,
-                   chunk_size, scale, workspace, workspace_bytes, stream);
+  Extras x;
+  x.ckpt = ckpt;
+  x.ckpt_interval = ckpt_interval;
+  return chunk_fwd(q, k, v, g, beta, h0, o, h_T, x, B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
+                   workspace_bytes, stream);
 }
 
 kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *z,
@@ -241,8 +293,66 @@ kda_status_t kda_chunk_fwd_gated(const void *q, const void *k, const void *v, co
                                  size_t workspace_bytes, kda_stream_t stream) {
   if (!(g_min >= -5.f && g_min < 0.f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
   if (B > 0 && H > 0 && T > 0 && !A_log) return KDA_ERR_INVALID_ARG;
-  return chunk_fwd(q, k, v, z, beta, h0, o, h_T, nullptr, 0, A_log, g_min, B, H, T, dk, dv, dtype, chunk_size, scale,
-                   workspace, workspace_bytes, stream);
+  Extras x;
+  x.A_log = A_log;
+  x.g_min = g_min;
+  return chunk_fwd(q, k, v, z, beta, h0, o, h_T, x, B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
+                   workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_fwd_outgate(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                                   const float *h0, const void *gate, const float *rms_weight, float eps, void *y,
+                                   float *h_T, int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                   int chunk_size, float scale, void *workspace, size_t workspace_bytes,
+                                   kda_stream_t stream) {
+  if (!(eps >= 0.f) || !isfinite(eps)) return KDA_ERR_INVALID_ARG;
+  if (B > 0 && H > 0 && T > 0 && (!gate || !rms_weight)) return KDA_ERR_INVALID_ARG;
+  Extras x;
+  x.gate = (B > 0 && H > 0 && T > 0) ? gate : nullptr;
+  x.rms_w = rms_weight;
+  x.eps = eps;
+  return chunk_fwd(q, k, v, g, beta, h0, y, h_T, x, B, H, T, dk, dv, dtype, chunk_size, scale, workspace,
+                   workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_transition(const void *k, const void *v, const void *g, const void *beta, float *St,
+                                  float *M, int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                  kda_stream_t stream) {
+  if (B < 0 || H < 0 || T < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
+  if ((int64_t)B * H > (int64_t)INT32_MAX / 2) return KDA_ERR_SHAPE;
+  // the transition-only kernel is the tensor-core one
+  if (dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (dk != 128 || dv != 128) return KDA_ERR_SHAPE;
+  const size_t n = (size_t)B * H;
+  if (n == 0) return KDA_OK;
+  if (!St || !M || (T > 0 && (!k || !v || !g || !beta))) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {T > 0 ? k : nullptr, T > 0 ? v : nullptr, T > 0 ? g : nullptr, St, M};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+  if (T > 0 && ((uintptr_t)beta & 1u) != 0) return KDA_ERR_ALIGNMENT;
+  const size_t e = 2;
+  const Range rk = range_of(k, n * T * dk * e), rv = range_of(v, n * T * dv * e), rg = range_of(g, n * T * dk * e),
+              rb = range_of(beta, n * T * e), rs = range_of(St, n * dk * dv * 4), rm = range_of(M, n * dk * dk * 4);
+  const Range ins[] = {rk, rv, rg, rb};
+  for (const Range &r : ins)
+    if (overlap(rs, r) || overlap(rm, r)) return KDA_ERR_ALIAS;
+  if (overlap(rs, rm)) return KDA_ERR_ALIAS;
+  kda_status_t st = check_device();
+  if (st != KDA_OK) return st;
+  kda::ChunkArgs a;
+  memset(&a, 0, sizeof(a));
+  a.k = k; a.v = v; a.g = g; a.beta = beta;
+  a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv;
+  a.bf16 = 1;
+  a.scale = 1.f;
+  a.status = kda::device_status_ptr();
+  a.segments = 1;
+  a.wait_ns = kda::debug_wait_ns();
+  a.stall = kda::debug_stall();
+  if (!a.status) return KDA_ERR_CUDA;
+  return kda::launch_chunk_tc32_transition(a, St, M, (cudaStream_t)stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_weight, float eps, void *y,
@@ -360,6 +470,16 @@ kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, con
   a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
   const cudaError_t ce = kda::launch_recurrent_step(a, (cudaStream_t)stream);
   return ce == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_debug_set_wait_limit(unsigned long long ns) {
+  kda::g_wait_ns.store(ns == 0 ? kda::kDefaultWaitNs : (uint64_t)ns, std::memory_order_relaxed);
+  return KDA_OK;
+}
+
+kda_status_t kda_debug_inject_stall(int on) {
+  kda::g_stall.store(on ? 1 : 0, std::memory_order_relaxed);
+  return KDA_OK;
 }
 
 kda_status_t kda_get_device_status(kda_stream_t stream) {

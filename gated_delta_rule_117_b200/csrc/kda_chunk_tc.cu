@@ -53,6 +53,7 @@
 // bounded; a wait that gives up sets the device status word and the whole CTA
 // drains without further MMAs.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "kda_internal.cuh"
 #include "kda_tmap.cuh"
@@ -92,17 +93,24 @@ constexpr int kXa = 204096;      // fp32 [32][33]: Qs_lo Kc_hi part of A
 constexpr int kFac = 208320;     // [3]: fp32 e^rho[128], e^{G_31-rho}[128] (1 KB each)
 constexpr int kXch = 212928;     // fp32 [2][128]: per-half sums of g (16 tokens each)
 constexpr int kBeta = 213952;    // [2]: fp32 beta[32] (written by token A, read by token B)
-constexpr int kBar = 214208;     // mbarriers
-constexpr int kMisc = 214336;    // TMEM base address, abort flag
+constexpr int kBar = 214208;     // mbarriers (32 slots)
+constexpr int kMisc = 214464;    // TMEM base address, abort flag
 constexpr int kOst = 215040;     // output tile staged for the TMA store: o h0 | o h1 (4 KB each)
 constexpr int kSmemBytes = 223232 + 1024;
+// Fused Eq. 6 output edge only: per-token partial sums of squares [4 warps][32
+// tokens] (row 0 then holds 1 / rms), and the chunk's output-gate tile (TMA).
+constexpr int kPart = 214528;
+constexpr int kGateT = 223232;
+constexpr int kSmemBytesOut = kGateT + 8192 + 1024;
+static_assert(kMisc + 8 <= kPart && kPart + 512 <= kOst && kGateT % 1024 == 0 && kSmemBytesOut <= 232448,
+              "output-edge smem layout");
 // each region ends where the next begins (or before)
 static_assert(kRawQK + 16384 <= kRawG && kRawG + 8192 <= kRawV && kRawV + 8192 <= kQKW, "smem layout");
 static_assert(kQKW + 2 * 32768 <= kKC && kKC + 3 * 16384 <= kST && kST + 32768 <= kAH, "smem layout");
 static_assert(kVTL + 8192 <= kST + 32768 && kAH + 3 * 4096 <= kTT && kTT + 2048 <= kLf, "smem layout");
 static_assert(kLf + 4224 <= kNf && kNf + 4224 <= kXf && kXf + 16 * 17 * 4 <= kXa && kXa + 4224 <= kFac, "smem layout");
 static_assert(kFac + 3 * 1024 <= kXch && kXch + 2 * 128 * 4 <= kBeta && kBeta + 2 * 128 <= kBar, "smem layout");
-static_assert(kBar + 8 * 16 <= kMisc && kMisc + 8 <= kOst && kOst + 8192 + 1024 <= kSmemBytes, "smem layout");
+static_assert(kBar + 8 * 32 <= kMisc && kMisc + 8 <= kOst && kOst + 8192 + 1024 <= kSmemBytes, "smem layout");
 static_assert(kOst % 1024 == 0 && kQKW % 1024 == 0 && kKC % 1024 == 0 && kST % 1024 == 0, "swizzled tiles");
 static_assert(kAH % 512 == 0 && kTT % 512 == 0, "64-byte swizzled tiles");
 static_assert(kSmemBytes <= 232448, "over the per-CTA shared memory limit");
@@ -122,9 +130,12 @@ enum {
   B_DS,        // dS and O-intra MMAs done
   B_CD0,       // [2] the chain's [O | V~] MMAs of the chunk are done (tcgen05.commit)
   B_CD1,
+  B_DRAIN,     // every MMA issued by the three issuing warps is done (count 3; before TMEM is released)
+  B_GATE,      // the output-gate tile of the chunk landed (fused Eq. 6 edge; TMA)
+  B_NEVER,     // nothing arrives here: the wait of an injected stall (failure-detection tests)
   B_COUNT
 };
-static_assert(B_COUNT <= 16, "mbarrier region holds 16 barriers");
+static_assert(B_COUNT <= 32, "mbarrier region holds 32 barriers");
 
 // TMEM columns (fp32, 128 lanes).  The output and pseudo-value accumulators
 // of a chunk parity are adjacent ([O | U]) so one N = 64 MMA updates both.
@@ -164,6 +175,11 @@ struct TcParams {
   int nseg;
   int mode;
   float scale;
+  uint64_t wait_ns;  // wall-time limit of every wait (ns)
+  int stall;         // 1: the chain first waits on a barrier nothing arrives on (failure-detection tests)
+  const float *rms_w;  // [H][128] RMSNorm weights of the fused Eq. 6 edge (the gate map holds its gate)
+  float eps;
+  int m_rowmajor;  // transition runs: M stored row-major (1) or transposed for the segment scan (0)
 };
 
 struct Ctx {
@@ -171,16 +187,19 @@ struct Ctx {
   uint64_t *bar;
   volatile int *abort;
   unsigned *status;
+  uint64_t wait_ns;
 };
 
 // Bounded wait: sleeps on the barrier (no spinning), returns false as soon as
-// another role aborted, and gives up after 2 s of wall time.
-__device__ __forceinline__ bool wait_bar_loop(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status) {
+// another role aborted, and gives up after wait_ns of wall time (2 s unless a
+// test shortened it), recording the timeout in the device status word.
+__device__ __forceinline__ bool wait_bar_loop(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status,
+                                              uint64_t wait_ns) {
   const uint64_t t_start = global_ns();
   for (;;) {
     if (mbar_try_wait_sleep(b, parity, 1000000u)) return true;
     if (*abort) return false;
-    if (global_ns() - t_start > 2000000000ull) break;
+    if (global_ns() - t_start > wait_ns) break;
   }
   *abort = 1;
   atomicExch(status, kDevTimeout);
@@ -189,18 +208,19 @@ __device__ __forceinline__ bool wait_bar_loop(uint64_t *b, uint32_t parity, vola
 __device__ __forceinline__ bool wait_bar(const Ctx &x, int slot, uint32_t parity) {
   uint64_t *b = &x.bar[slot];
   if (mbar_try_wait(b, parity)) return true;
-  return wait_bar_loop(b, parity, x.abort, x.status);
+  return wait_bar_loop(b, parity, x.abort, x.status, x.wait_ns);
 }
 // The token warpgroups share one out-of-line copy of the sleeping loop (their
 // instruction streams compete for each sub-partition's instruction cache).  The
 // chain cannot call: a call inside its 248-register region fails allocation.
-__device__ __noinline__ bool wait_bar_slow(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status) {
-  return wait_bar_loop(b, parity, abort, status);
+__device__ __noinline__ bool wait_bar_slow(uint64_t *b, uint32_t parity, volatile int *abort, unsigned *status,
+                                           uint64_t wait_ns) {
+  return wait_bar_loop(b, parity, abort, status, wait_ns);
 }
 __device__ __forceinline__ bool wait_tok(const Ctx &x, int slot, uint32_t parity) {
   uint64_t *b = &x.bar[slot];
   if (mbar_try_wait(b, parity)) return true;
-  return wait_bar_slow(b, parity, x.abort, x.status);
+  return wait_bar_slow(b, parity, x.abort, x.status, x.wait_ns);
 }
 
 // hi/lo pair of (a, b): returns packed hi, writes packed lo.
@@ -223,7 +243,7 @@ __device__ __forceinline__ uint32_t split2(float a, float b, uint32_t &lo) {
 // memory loads are issued before the previous group's stores, so the loop
 // stays rolled (three warpgroups share each sub-partition's instruction
 // cache) without serialising on load latency.
-template <bool kGate>
+template <bool kGate, bool kNoQ>
 __device__ __forceinline__ void decay_group(const uint32_t (&gr)[4], const uint32_t (&qr)[4], const uint32_t (&kr)[4],
                                             float2 &R, bool fwd, unsigned char *qkw, unsigned char *kc,
                                             const uint32_t (&off)[4], float2 eA, float g_min, int row0, int nvalid) {
@@ -236,27 +256,31 @@ __device__ __forceinline__ void decay_group(const uint32_t (&gr)[4], const uint3
       // rows past the end of the sequence (zero-filled z) must not decay: g = 0 there
       if ((fwd ? row0 + u : row0 - u) >= nvalid) g = make_float2(0.f, 0.f);
     }
-    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr[u]));
     const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr[u]));
     const float2 Rn = __fadd2_rn(R, g);
     const float2 xr = fwd ? Rn : make_float2(-R.x, -R.y);
     R = Rn;
     const float x0 = fminf(fmaxf(xr.x, -87.f), 87.f), x1 = fminf(fmaxf(xr.y, -87.f), 87.f);
     const float2 ep = make_float2(__expf(x0), __expf(x1)), en = make_float2(__expf(-x0), __expf(-x1));
-    const float2 qe = __fmul2_rn(q, ep), ke = __fmul2_rn(k, ep), ki = __fmul2_rn(k, en);
-    uint32_t qlo, clo;
-    const uint32_t qhi = split2(qe.x, qe.y, qlo);
+    const float2 ke = __fmul2_rn(k, ep), ki = __fmul2_rn(k, en);
+    if (!kNoQ) {  // Qs hi/lo: only runs that write outputs need them
+      const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr[u]));
+      const float2 qe = __fmul2_rn(q, ep);
+      uint32_t qlo;
+      const uint32_t qhi = split2(qe.x, qe.y, qlo);
+      *reinterpret_cast<uint32_t *>(qkw + 4096 + off[u]) = qlo;
+      *reinterpret_cast<uint32_t *>(qkw + 8192 + off[u]) = qhi;
+    }
+    uint32_t clo;
     const __nv_bfloat162 khi = __float22bfloat162_rn(ke);
     const uint32_t chi = split2(ki.x, ki.y, clo);
     *reinterpret_cast<__nv_bfloat162 *>(qkw + off[u]) = khi;
-    *reinterpret_cast<uint32_t *>(qkw + 4096 + off[u]) = qlo;
-    *reinterpret_cast<uint32_t *>(qkw + 8192 + off[u]) = qhi;
     *reinterpret_cast<uint32_t *>(kc + off[u]) = chi;
     *reinterpret_cast<uint32_t *>(kc + 4096 + off[u]) = clo;
   }
 }
 
-template <bool kGate>
+template <bool kGate, bool kNoQ>
 __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs, float2 eA, float g_min, int nvalid) {
   unsigned char *sm = x.sm;
   const int pp = tt & 63, hf = tt >> 6;
@@ -274,7 +298,7 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs,
   for (int u = 0; u < 4; ++u) {
     o0[u] = sw128_off(row(u), cc);
     g0[u] = *reinterpret_cast<const uint32_t *>(rg + o0[u]);
-    q0[u] = *reinterpret_cast<const uint32_t *>(rq + o0[u]);
+    q0[u] = kNoQ ? 0u : *reinterpret_cast<const uint32_t *>(rq + o0[u]);
     k0[u] = *reinterpret_cast<const uint32_t *>(rk + o0[u]);
   }
   float2 R = make_float2(0.f, 0.f);
@@ -286,11 +310,11 @@ __device__ __forceinline__ void token_decay(const Ctx &x, int tt, int p, int fs,
       for (int u = 0; u < 4; ++u) {
         o1[u] = sw128_off(row(4 * grp + 4 + u), cc);
         g1[u] = *reinterpret_cast<const uint32_t *>(rg + o1[u]);
-        q1[u] = *reinterpret_cast<const uint32_t *>(rq + o1[u]);
+        q1[u] = kNoQ ? 0u : *reinterpret_cast<const uint32_t *>(rq + o1[u]);
         k1[u] = *reinterpret_cast<const uint32_t *>(rk + o1[u]);
       }
     }
-    decay_group<kGate>(g0, q0, k0, R, fwd, qkw, kc, o0, eA, g_min, row(4 * grp), nvalid);
+    decay_group<kGate, kNoQ>(g0, q0, k0, R, fwd, qkw, kc, o0, eA, g_min, row(4 * grp), nvalid);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       g0[u] = g1[u];
@@ -416,13 +440,20 @@ __device__ __forceinline__ void store_st32(unsigned char *__restrict__ st, const
 }
 
 // kCkpt: the instantiation that can emit prefix-cache checkpoints; kGate: the
-// one whose g input holds the Eq. 5 logits z.  The plain one compiles without
-// either, so its register allocation is untouched.
-template <bool kCkpt, bool kGate>
+// one whose g input holds the Eq. 5 logits z; kTrans: the segment-transition
+// runs of in-device context parallelism, which write no output, so they skip
+// everything only the output needs (the q-side operands Qs, the A tile, the O
+// products; the M run, whose v is zero, also skips the U product).  The plain
+// one compiles without any of these, so its register allocation is untouched.
+// kOut: the instantiation with the report's Eq. 6 output edge fused into the
+// output epilogue: it writes y = Sigmoid(gate) * RMSNorm_w(o) (per token and
+// head, over dv) instead of o, so o never reaches memory.
+template <bool kCkpt, bool kGate, bool kTrans, bool kOut>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mg,
-                    const __grid_constant__ CUtensorMap mo, const TcParams p) {
+                    const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mgate,
+                    const TcParams p) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   // 1024-byte aligned base, derived by pointer arithmetic so that every access
   // through it stays a shared-memory (not generic) access.
@@ -432,6 +463,7 @@ __global__ void __launch_bounds__(NT, 1)
   x.bar = reinterpret_cast<uint64_t *>(sm + kBar);
   x.abort = reinterpret_cast<volatile int *>(sm + kMisc + 4);
   x.status = p.status;
+  x.wait_ns = p.wait_ns;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kMisc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -450,8 +482,8 @@ __global__ void __launch_bounds__(NT, 1)
   const int tb = seg * p.seg_len;
   const int te = min(T, tb + p.seg_len);
   const int nchunks = (te - tb + C - 1) / C;
-  const bool v_zero = kind == 2;
-  const bool store_o = p.mode != kModeSegTransition;
+  const bool v_zero = kTrans && kind == 2;
+  const bool store_o = !kTrans;
   const float *h0src = nullptr;
   float *hdst = nullptr;
   if (p.mode == kModeChain) {
@@ -467,7 +499,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sbase = smem_u32(sm);
 
   if (tid == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(&x.bar[i], 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&x.bar[i], i == B_DRAIN ? 3u : 1u);
     *x.abort = 0;
     mbar_init_fence();
   }
@@ -504,12 +536,21 @@ __global__ void __launch_bounds__(NT, 1)
       const uint64_t dS = sdesc_sw128(sbase + kST, 16, 1024);
       const uint64_t dB = sdesc_sw128(sbase + kQKW + pb * 32768 + 8192, 16, 1024);  // rows: Qs, -W~
       const uint32_t tO = tbase + tOU(t % 3);
-      mma_bf16_warp(tO, dS, dB, idO, false);
-      mma_bf16_warp(tO + 32, dS, sdesc_add(dB, 4096), idO, true);
+      if (kTrans) {
+        // V~ alone (rows -W~), onto U; the M run has no U (v = 0) and starts from zero
 #pragma unroll 1
-      for (int ks = 1; ks < 8; ++ks) {  // rolled: MMA issue loops are kept small for the instruction cache
-        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-        mma_bf16_warp(tO, sdesc_add(dS, koff), sdesc_add(dB, koff), idOU, true);
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_warp(tO + 32, sdesc_add(dS, koff), sdesc_add(dB, 4096 + koff), idO, ks > 0 || !v_zero);
+        }
+      } else {
+        mma_bf16_warp(tO, dS, dB, idO, false);
+        mma_bf16_warp(tO + 32, dS, sdesc_add(dB, 4096), idO, true);
+#pragma unroll 1
+        for (int ks = 1; ks < 8; ++ks) {  // rolled: MMA issue loops are kept small for the instruction cache
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_warp(tO, sdesc_add(dS, koff), sdesc_add(dB, koff), idOU, true);
+        }
       }
       mma_commit_warp(&x.bar[B_V1]);
       // these MMAs are the last readers of the chunk's double-buffered operands
@@ -517,7 +558,21 @@ __global__ void __launch_bounds__(NT, 1)
       // two chunks behind, so the buffers of parity pb may take chunk t + 2
       mma_commit_warp(&x.bar[B_CD0 + pb]);
     };
+    // fused Eq. 6 edge: this thread's RMSNorm weight; the gate tile of chunk 0
+    float wgt = 0.f;
+    int gate_issued = -1;  // last chunk whose gate tile was requested (abort path)
+    if (kOut) {
+      wgt = p.rms_w[(size_t)(bh % p.H) * D + e];
+      if (warp == 0 && nchunks > 0) {
+        mbar_arrive_expect_tx_warp(&x.bar[B_GATE], 2 * 4096);
+        tma_load_3d_warp(sm + kGateT, &mgate, &x.bar[B_GATE], 0, tb, bh);
+        tma_load_3d_warp(sm + kGateT + 4096, &mgate, &x.bar[B_GATE], 64, tb, bh);
+        gate_issued = 0;
+      }
+    }
     if (nchunks > 0) {
+      // injected stall: a wait that can only end by giving up, which aborts the CTA
+      if (p.stall) wait_bar(x, B_NEVER, 0u);
       const bool ready = wait_bar(x, B_WT0, 0u);
       const float2 *erho = reinterpret_cast<const float2 *>(sm + kFac);
 #pragma unroll
@@ -570,7 +625,7 @@ __global__ void __launch_bounds__(NT, 1)
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = sdesc_add(aB, ks * 32);
             mma_bf16_warp(tbase + tDS, ad, sdesc_add(kB, ks * 2048), idS, part > 0 || ks > 0);
-            mma_bf16_warp(tbase + tOU(t % 3), ad, sdesc_add(mB, ks * 32), idO, true);
+            if (!kTrans) mma_bf16_warp(tbase + tOU(t % 3), ad, sdesc_add(mB, ks * 32), idO, true);
           }
         }
         mma_commit_warp(&x.bar[B_DS]);
@@ -641,14 +696,61 @@ __global__ void __launch_bounds__(NT, 1)
       // (rows past the end of the sequence are clipped by the tensor map)
       if (store_o) {
         unsigned char *ot = sm + kOst + (e >> 6) * 4096;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          float ov[16];
-          tmem_ld16(tl + tOU(t % 3) + 16 * hh, ov);
+        if (kOut) {
+          // Eq. 6 edge: y[r][e] = Sigmoid(gate[r][e]) w[e] o[r][e] / rms(o[r]), the rms
+          // over the 128 channels, i.e. across the four chain warps
+          float ov[32], v[32];
+          tmem_ld32(tl + tOU(t % 3), ov);
           tmem_ld_wait(ov);
 #pragma unroll
-          for (int r = 0; r < 16; ++r)
-            *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(16 * hh + r, e & 63)) = __float2bfloat16_rn(p.scale * ov[r]);
+          for (int r = 0; r < 32; ++r) {
+            ov[r] *= p.scale;
+            v[r] = ov[r] * ov[r];
+          }
+          // butterfly over the warp: lane r ends with the sum over the warp's 32 channels for token r
+#pragma unroll
+          for (int k = 16; k >= 1; k >>= 1) {
+            const bool up = (lane & k) != 0;
+#pragma unroll
+            for (int i = 0; i < k; ++i) {
+              const float send = up ? v[i] : v[i + k];
+              const float keep = up ? v[i + k] : v[i];
+              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+            }
+          }
+          float *part = reinterpret_cast<float *>(sm + kPart);
+          part[warp * 32 + lane] = v[0];
+          named_sync(kBarChain, 128);
+          if (warp == 0) {
+            const float ssq = (part[lane] + part[32 + lane]) + (part[64 + lane] + part[96 + lane]);
+            part[lane] = rsqrtf(ssq * (1.f / D) + p.eps);  // 1 / rms of token `lane`
+          }
+          wait_bar(x, B_GATE, (uint32_t)t & 1u);
+          named_sync(kBarChain, 128);
+          const unsigned char *gtile = sm + kGateT + (e >> 6) * 4096;
+          const float4 *rin4 = reinterpret_cast<const float4 *>(part);
+#pragma unroll
+          for (int r4 = 0; r4 < 8; ++r4) {
+            const float4 ri = rin4[r4];
+            const float rr[4] = {ri.x * wgt, ri.y * wgt, ri.z * wgt, ri.w * wgt};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int r = 4 * r4 + u;
+              const float gv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gtile + sw128_off(r, e & 63)));
+              const float sg = __fdividef(1.f, 1.f + __expf(-gv));
+              *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(r, e & 63)) = __float2bfloat16_rn(ov[r] * rr[u] * sg);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            float ov[16];
+            tmem_ld16(tl + tOU(t % 3) + 16 * hh, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+              *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(16 * hh + r, e & 63)) = __float2bfloat16_rn(p.scale * ov[r]);
+          }
         }
         fence_proxy_async_smem();
         named_sync(kBarChain, 128);
@@ -657,6 +759,12 @@ __global__ void __launch_bounds__(NT, 1)
           tma_store_3d_warp(&mo, sm + kOst + 4096, 64, t0, bh);
           bulk_commit_warp();
           if (lane == 0) bulk_wait_read_all();  // the tile is rewritten next chunk
+          if (kOut && has_next && *x.abort == 0) {  // every thread has read this chunk's gate tile
+            mbar_arrive_expect_tx_warp(&x.bar[B_GATE], 2 * 4096);
+            tma_load_3d_warp(sm + kGateT, &mgate, &x.bar[B_GATE], 0, t0 + C, bh);
+            tma_load_3d_warp(sm + kGateT + 4096, &mgate, &x.bar[B_GATE], 64, t0 + C, bh);
+            gate_issued = t + 1;
+          }
         }
       }
       if (warp == 0 && !issued && __shfl_sync(0xffffffffu, wait_bar(x, wt_next, wt_par), 0)) issue_v1(t + 1);
@@ -664,7 +772,10 @@ __global__ void __launch_bounds__(NT, 1)
       if (!go) break;
     }
     if (warp == 0 && lane == 0) bulk_wait_all();
-    if (*x.abort == 0 && hdst && kind == 2) {
+    if (kOut && warp == 0 && lane == 0 && *x.abort && gate_issued >= 0)  // let the last gate copy land
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_GATE], (uint32_t)gate_issued & 1u); ++i) {
+      }
+    if (*x.abort == 0 && hdst && kind == 2 && !p.m_rowmajor) {
       // the segment transition is stored transposed (row e = column e of M) for the scan
       float4 *row = reinterpret_cast<float4 *>(hdst + (size_t)e * D);
 #pragma unroll
@@ -691,7 +802,7 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t idG = idesc_bf16(128, 64, false, false, false);
     // TMA issue, called by all of warp 4 (one elected lane issues).
     // transition runs write no outputs and need no q: its buffer stays zero
-    const bool need_q = store_o;
+    constexpr bool need_q = !kTrans;
     auto tma_qkg = [&](int t) {
       mbar_arrive_expect_tx_warp(&x.bar[B_QKG], (need_q ? 6 : 4) * 4096);
       const int y = tb + t * C;
@@ -704,11 +815,6 @@ __global__ void __launch_bounds__(NT, 1)
       tma_load_3d_warp(sm + kRawG, &mg, &x.bar[B_QKG], 0, y, bh);
       tma_load_3d_warp(sm + kRawG + 4096, &mg, &x.bar[B_QKG], 64, y, bh);
     };
-    if (!need_q) {
-      uint4 *zq = reinterpret_cast<uint4 *>(sm + kRawQK);
-      for (int i = tt; i < 512; i += 128) zq[i] = make_uint4(0, 0, 0, 0);
-      named_sync(kBarTokA, 128);
-    }
     int qkg_issued = -1;  // last chunk whose q, k, g copy was issued (abort path)
     if (warp == 5 && nchunks > 0) {
       if (lane == 0) {
@@ -730,7 +836,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (t >= 2) wait_tok(x, B_CD0 + pb, (uint32_t)((t - 2) >> 1) & 1u);  // chunk t-2's buffers are free
       const bool landed = wait_tok(x, B_QKG, (uint32_t)t & 1u);
       if (tt < C) reinterpret_cast<float *>(sm + kBeta + pb * 128)[tt] = __bfloat162float(__ushort_as_bfloat16(beta_cur));
-      token_decay<kGate>(x, tt, pb, t % 3, eA, p.g_min, te - t0);
+      token_decay<kGate, kTrans>(x, tt, pb, t % 3, eA, p.g_min, te - t0);
       fence_proxy_async_smem();
       const bool go = named_sync_and(kBarTokA, 128, *x.abort == 0);
       if (tt == 0) mbar_arrive(&x.bar[B_DEC0 + pb]);
@@ -766,7 +872,7 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tl = tbase + ((uint32_t)(32 * quarter) << 16);
     const uint32_t idMK = idesc_bf16(128, 32, true, false, false);
     auto tma_v = [&](int t) {
-      if (v_zero) return;  // transition runs: v = 0, the buffer holds zeros
+      if (v_zero) return;  // the M run: v = 0, no U product, nothing to load
       mbar_arrive_expect_tx_warp(&x.bar[B_V], 2 * 4096);
       tma_load_3d_warp(sm + kRawV, &mv, &x.bar[B_V], 0, tb + t * C, bh);
       tma_load_3d_warp(sm + kRawV + 4096, &mv, &x.bar[B_V], 64, tb + t * C, bh);
@@ -776,10 +882,6 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float *N = reinterpret_cast<float *>(sm + kNf);
       for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
-      if (v_zero) {  // v = 0 for a transition run: the U MMA then yields U = 0
-        uint4 *zv = reinterpret_cast<uint4 *>(sm + kRawV);
-        for (int i = tt; i < 512; i += 128) zv[i] = make_uint4(0, 0, 0, 0);
-      }
       named_sync(kBarTokB, 128);
     }
     int v_issued = -1;  // last chunk whose v copy was issued (abort path)
@@ -799,7 +901,7 @@ __global__ void __launch_bounds__(NT, 1)
       const uint32_t tg = (pb ? tG1 : tG0);
       float a[32];
       const int r = lane;
-      if (quarter == 0 || quarter == 2) {
+      if (quarter == 0 || (!kTrans && quarter == 2)) {
         float b[32];
         tmem_ld32(tl + tg, a);
         tmem_ld32(tl + tg + 32, b);
@@ -815,7 +917,7 @@ __global__ void __launch_bounds__(NT, 1)
           __syncwarp();
           solve_diag_blocks(x, lane);
         }
-      } else if (quarter == 1) {
+      } else if (!kTrans && quarter == 1) {
         tmem_ld32(tl + tg, a);
         tmem_ld_wait(a);
         float *Xa = reinterpret_cast<float *>(sm + kXa);
@@ -824,7 +926,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tc_fence_before();
       named_sync(kBarTokB, 128);
-      if (quarter == 2) {
+      if (!kTrans && quarter == 2) {
         const float *Xa = reinterpret_cast<const float *>(sm + kXa);
         unsigned char *ah = sm + kAH + (t % 3) * 4096;
 #pragma unroll
@@ -859,7 +961,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t bd = sdesc_add(dT, ks * 32);
-            mma_bf16_warp(tbase + tOU(t % 3) + 32, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
+            if (!v_zero) mma_bf16_warp(tbase + tOU(t % 3) + 32, sdesc_add(dV, ks * 2048), bd, idMK, ks > 0);
             mma_bf16_warp(tbase + tW, sdesc_add(dKs, ks * 2048), bd, idMK, ks > 0);
           }
           mma_commit_warp(&x.bar[B_UW]);
@@ -893,16 +995,19 @@ __global__ void __launch_bounds__(NT, 1)
       }
   }
 
+  // Drain: each MMA-issuing warp (chain warp 0, token warps 4 and 8) commits
+  // once more to B_DRAIN, which completes when every MMA those warps issued has
+  // completed -- also after an abort, when some were never waited for.  TMEM is
+  // released only then.  (The TMA loads were drained by their roles above and
+  // the output stores by the chain's bulk wait.)
+  if (warp == 0 || warp == 4 || warp == 8) mma_commit_warp(&x.bar[B_DRAIN]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 4) {
-    // after an abort an MMA issued before it may still be running: give it
-    // time to retire before its TMEM is released
-    if (*x.abort) {
-      const uint64_t t_start = global_ns();
-      while (global_ns() - t_start < 200000ull) __nanosleep(10000);
-    }
+    bool drained = false;
+    for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(&x.bar[B_DRAIN], 0u);
+    if (!drained) atomicExch(x.status, kDevTimeout);
     __syncwarp();
     tmem_dealloc(tbase, kTmemCols);
   }
@@ -1001,14 +1106,19 @@ size_t tc32_workspace(int BH, int T) {
 
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   if (a.B * a.H == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mg;
+  CUtensorMap mq, mk, mv, mg, mo, mgate;
   const int BH = a.B * a.H;
   const uint64_t T = (uint64_t)(a.T > 0 ? a.T : 1), n = (uint64_t)BH;
-  CUtensorMap mo;
   if (!encode_tmap_bf16_3d(&mq, a.q, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mk, a.k, D, T, n, 64, C) ||
       !encode_tmap_bf16_3d(&mv, a.v, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mg, a.g, D, T, n, 64, C) ||
       !encode_tmap_bf16_3d(&mo, a.o, D, T, n, 64, C))
     return cudaErrorInvalidValue;
+  const bool out_edge = a.gate != nullptr;
+  if (out_edge) {
+    if (!encode_tmap_bf16_3d(&mgate, a.gate, D, T, n, 64, C)) return cudaErrorInvalidValue;
+  } else {
+    mgate = mq;  // not read
+  }
   TcParams p;
   p.beta = (const __nv_bfloat16 *)a.beta;
   p.h0 = a.h0;
@@ -1025,26 +1135,47 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.A_log = a.A_log;
   p.g_min = a.g_min;
   p.H = a.H;
+  p.wait_ns = a.wait_ns;
+  p.stall = a.stall;
+  p.rms_w = a.rms_w;
+  p.eps = a.eps;
+  p.m_rowmajor = 0;
   const bool gated = a.A_log != nullptr;
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_tc_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  // one variant per call: checkpoints, the fused gate and the fused output edge do not combine
+  if ((p.ckpt != nullptr) + (int)gated + (int)out_edge > 1) return cudaErrorInvalidValue;
+  cudaError_t e = cudaSuccess;
+  {
+    // every instantiation the launches below may use
+    const void *fns[] = {(const void *)chunk_tc_kernel<false, false, false, false>,
+                         (const void *)chunk_tc_kernel<true, false, false, false>,
+                         (const void *)chunk_tc_kernel<false, true, false, false>,
+                         (const void *)chunk_tc_kernel<false, false, true, false>,
+                         (const void *)chunk_tc_kernel<false, true, true, false>};
+    for (const void *f : fns)
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute((const void *)chunk_tc_kernel<false, false, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytesOut);
+  }
   if (e != cudaSuccess) return e;
+  // the run that writes outputs: the chain (unsegmented) or the final pass
+  auto launch_out = [&](int grid) {
+    if (p.ckpt)
+      chunk_tc_kernel<true, false, false, false><<<grid, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    else if (gated)
+      chunk_tc_kernel<false, true, false, false><<<grid, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    else if (out_edge)
+      chunk_tc_kernel<false, false, false, true><<<grid, NT, kSmemBytesOut, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    else
+      chunk_tc_kernel<false, false, false, false><<<grid, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    return cudaGetLastError();
+  };
   const int P = a.segments > 1 ? a.segments : 1;
   if (P == 1) {
     p.seg_len = a.T > 0 ? a.T : 1;
     p.nseg = 1;
     p.mode = kModeChain;
-    if (p.ckpt)
-      chunk_tc_kernel<true, false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
-    else if (gated)
-      chunk_tc_kernel<false, true><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
-    else
-      chunk_tc_kernel<false, false><<<BH, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
-    return cudaGetLastError();
+    return launch_out(BH);
   }
   const size_t mat = (size_t)D * D;
   float *ws = static_cast<float *>(a.workspace);
@@ -1061,9 +1192,9 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   float *const ckpt = p.ckpt;
   p.ckpt = nullptr;  // transition runs start from 0 or I: no checkpoints there
   if (gated)
-    chunk_tc_kernel<false, true><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    chunk_tc_kernel<false, true, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
   else
-    chunk_tc_kernel<false, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+    chunk_tc_kernel<false, false, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
@@ -1072,12 +1203,42 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.mode = kModeSegFinal;
   p.ckpt = ckpt;
-  if (p.ckpt)
-    chunk_tc_kernel<true, false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
-  else if (gated)
-    chunk_tc_kernel<false, true><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
-  else
-    chunk_tc_kernel<false, false><<<BH * P, NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, p);
+  return launch_out(BH * P);
+}
+
+cudaError_t launch_chunk_tc32_transition(const ChunkArgs &a, float *St, float *M, cudaStream_t st) {
+  if (a.B * a.H == 0) return cudaSuccess;
+  const int BH = a.B * a.H;
+  const uint64_t T = (uint64_t)(a.T > 0 ? a.T : 1), n = (uint64_t)BH;
+  // with no token the maps are never read; any valid device address serves as their base
+  const void *kb = a.T > 0 ? a.k : (const void *)St, *vb = a.T > 0 ? a.v : (const void *)St,
+             *gb = a.T > 0 ? a.g : (const void *)St;
+  CUtensorMap mk, mv, mg;
+  if (!encode_tmap_bf16_3d(&mk, kb, D, T, n, 64, C) || !encode_tmap_bf16_3d(&mv, vb, D, T, n, 64, C) ||
+      !encode_tmap_bf16_3d(&mg, gb, D, T, n, 64, C))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  p.beta = (const __nv_bfloat16 *)a.beta;
+  p.status = a.status;
+  p.m_out = M;
+  p.st_out = St;
+  p.T = a.T;
+  p.scale = 1.f;
+  p.ckpt_interval = 1;
+  p.H = a.H;
+  p.wait_ns = a.wait_ns;
+  p.stall = a.stall;
+  p.m_rowmajor = 1;
+  // every chain is one segment whose transition is wanted: two CTAs per chain
+  // (state from zero; state from I with v = 0), no final pass
+  p.mode = kModeSegTransition;
+  p.nseg = 2;
+  p.seg_len = a.T;
+  cudaError_t e = cudaFuncSetAttribute((const void *)chunk_tc_kernel<false, false, true, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  chunk_tc_kernel<false, false, true, false><<<BH * 2, NT, kSmemBytes, st>>>(mk, mk, mv, mg, mk, mk, p);
   return cudaGetLastError();
 }
 

@@ -29,7 +29,16 @@ struct ChunkArgs {
   int n_ckpt;         // T / ckpt_interval
   const float *A_log;  // [H][dk] decay log-scales when `g` holds the logits z (fused Eq. 5 gate), else null
   float g_min;         // lower bound of the fused gate
+  uint64_t wait_ns;    // wall-time limit of the tensor-core kernel's bounded waits
+  int stall;           // failure-detection tests: make a wait run out (kda_debug_inject_stall)
+  const void *gate;    // [B][H][T][dv] output gate of the fused Eq. 6 edge (o then holds y), or null
+  const float *rms_w;  // [H][dv] RMSNorm weights of that edge
+  float eps;
 };
+
+// Failure-detection test settings (kda_debug_set_wait_limit, kda_debug_inject_stall).
+uint64_t debug_wait_ns();
+int debug_stall();
 
 struct DecodeArgs {
   const void *q, *k, *v, *g, *beta;
@@ -65,6 +74,9 @@ cudaError_t launch_kcp_compose(const float *M, const float *St, const float *h0,
                                int dv, cudaStream_t s);
 cudaError_t launch_chunk_simt16(const ChunkArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t s);
+// Segment transition of every chain over its T tokens (kda_chunk_transition):
+// St [BH][128][128] the end state from zero, M [BH][128][128] row-major.
+cudaError_t launch_chunk_tc32_transition(const ChunkArgs &a, float *St, float *M, cudaStream_t s);
 // Planning of the tensor-core path: segments per chain, segment length, workspace bytes.
 void tc32_plan(int BH, int T, int *segments, int *seg_len);
 int tc32_segments(int BH, int T);

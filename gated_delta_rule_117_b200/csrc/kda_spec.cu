@@ -13,7 +13,11 @@
 // Each token is the decode step of Eq. 1 (same thread layout as the decode
 // kernel: rows of S in registers as float4, column sums over dk reduced
 // through shared memory), so the window costs one read and at most one write
-// of the state instead of one of each per token.
+// of the state instead of one of each per token.  The window's inputs are
+// staged in shared memory once (in blocks of WB tokens) while the state load
+// is in flight; the column partial sums are double-buffered by token parity,
+// so each token costs one barrier; the q-side sums are formed only for the
+// tokens whose output is verified.
 #include <cuda_bf16.h>
 
 #include "kda_internal.cuh"
@@ -32,7 +36,11 @@ struct SpecShape {
   static constexpr int RP = (DK < 256 / TPR) ? DK : 256 / TPR;   // row groups
   static constexpr int NT = TPR * RP;                            // threads per CTA
   static constexpr int RPT = DK / RP;                            // rows per thread
+  static constexpr int WB = 8;                                   // window tokens staged at a time
 };
+
+__device__ __forceinline__ float2 lo2(float4 a) { return make_float2(a.x, a.y); }
+__device__ __forceinline__ float2 hi2(float4 a) { return make_float2(a.z, a.w); }
 
 template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
@@ -40,83 +48,103 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
                               const TIn *__restrict__ g, const TIn *__restrict__ beta, float *S,
                               TIn *__restrict__ o, const int *__restrict__ n_replay, int H, int W, float scale) {
   using Sh = SpecShape<DK, DV>;
-  constexpr int TPR = Sh::TPR, RP = Sh::RP, NT = Sh::NT, RPT = Sh::RPT;
+  constexpr int TPR = Sh::TPR, RP = Sh::RP, NT = Sh::NT, RPT = Sh::RPT, WB = Sh::WB;
   const int bh = blockIdx.x;
   const int tid = threadIdx.x;
   const int tx = tid % TPR, ty = tid / TPR;
-  __shared__ float sk[DK], sq[DK], sa[DK], sv[DV];
-  __shared__ float4 red_p[RP][TPR], red_r[RP][TPR];
-  __shared__ float s_qk, s_b;
+  // a block of up to WB window tokens, staged once: k, q, alpha = exp(g), v, beta, q.k
+  __shared__ float sk[WB][DK], sq[WB][DK], sa[WB][DK], sv[WB][DV], sb[WB], sqk[WB];
+  // column partial sums, double-buffered by token parity: one barrier per token
+  __shared__ float4 red_p[2][RP][TPR], red_r[2][RP][TPR];
 
   const int nr = min(max(n_replay[bh / H], 0), W);
   float4 *S4 = reinterpret_cast<float4 *>(S + (size_t)bh * DK * DV);
   float4 s[RPT];
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) s[r] = S4[(ty + r * RP) * TPR + tx];
+  for (int r = 0; r < RPT; ++r) s[r] = S4[(ty + r * RP) * TPR + tx];  // in flight while the window is staged
 
-  for (int t = 0; t < W; ++t) {
-    const size_t in_k = ((size_t)bh * W + t) * DK, in_v = ((size_t)bh * W + t) * DV;
-    for (int i = tid; i < DK; i += NT) {
-      sk[i] = to_f(k[in_k + i]);
-      sq[i] = to_f(q[in_k + i]);
-      sa[i] = expf(to_f(g[in_k + i]));
+  for (int t0 = 0; t0 < W; t0 += WB) {
+    const int nb = min(WB, W - t0);
+    if (t0 > 0) __syncthreads();  // the previous block's staged inputs are consumed
+    for (int e = tid; e < nb * DK; e += NT) {
+      const int u = e / DK, i = e % DK;
+      const size_t in = ((size_t)bh * W + t0 + u) * DK + i;
+      sk[u][i] = to_f(k[in]);
+      sq[u][i] = to_f(q[in]);
+      sa[u][i] = expf(to_f(g[in]));
     }
-    for (int j = tid; j < DV; j += NT) sv[j] = to_f(v[in_v + j]);
-    if (tid == 0) s_b = to_f(beta[(size_t)bh * W + t]);
+    for (int e = tid; e < nb * DV; e += NT) {
+      const int u = e / DV, j = e % DV;
+      sv[u][j] = to_f(v[((size_t)bh * W + t0 + u) * DV + j]);
+    }
+    if (tid < nb) sb[tid] = to_f(beta[(size_t)bh * W + t0 + tid]);
     __syncthreads();
-    const bool out = t >= nr;
-    if (out && tid < 32) {  // q . k, one warp
+    // q . k of each staged token: one warp per token
+    for (int u = tid >> 5; u < nb; u += NT / 32) {
       float acc = 0.f;
-      for (int i = tid; i < DK; i += 32) acc += sq[i] * sk[i];
+      for (int i = tid & 31; i < DK; i += 32) acc += sq[u][i] * sk[u][i];
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (tid == 0) s_qk = acc;
+      if ((tid & 31) == 0) sqk[u] = acc;
     }
-    float4 p = make_float4(0.f, 0.f, 0.f, 0.f), rr = p;
+    // (sqk is read after the first token's barrier below)
+    for (int u = 0; u < nb; ++u) {
+      const int t = t0 + u, par = t & 1;
+      const bool out = t >= nr;  // bonus / draft token: its output is verified
+      float2 p0 = make_float2(0.f, 0.f), p1 = p0, r0 = p0, r1 = p0;
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const int i = ty + r * RP;
-      const float a = sa[i], ka = sk[i], qa = sq[i];
-      s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
-      p.x += ka * s[r].x; p.y += ka * s[r].y; p.z += ka * s[r].z; p.w += ka * s[r].w;
-      rr.x += qa * s[r].x; rr.y += qa * s[r].y; rr.z += qa * s[r].z; rr.w += qa * s[r].w;
-    }
-    red_p[ty][tx] = p;
-    red_r[ty][tx] = rr;
-    __syncthreads();
-    float4 P = red_p[0][tx];
-#pragma unroll
-    for (int y = 1; y < RP; ++y) {
-      const float4 c = red_p[y][tx];
-      P.x += c.x; P.y += c.y; P.z += c.z; P.w += c.w;
-    }
-    const int j0 = 4 * tx;
-    const float b = s_b;
-    const float4 u = make_float4(b * (sv[j0 + 0] - P.x), b * (sv[j0 + 1] - P.y), b * (sv[j0 + 2] - P.z),
-                                 b * (sv[j0 + 3] - P.w));
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const float ki = sk[ty + r * RP];
-      s[r].x += ki * u.x; s[r].y += ki * u.y; s[r].z += ki * u.z; s[r].w += ki * u.w;
-    }
-    if (t == nr - 1)  // the last accepted token: this state is committed
-#pragma unroll
-      for (int r = 0; r < RPT; ++r) S4[(ty + r * RP) * TPR + tx] = s[r];
-    if (out && ty == 0) {
-      float4 R = red_r[0][tx];
+      for (int r = 0; r < RPT; ++r) {
+        const int i = ty + r * RP;
+        const float2 a = make_float2(sa[u][i], sa[u][i]), ka = make_float2(sk[u][i], sk[u][i]);
+        float2 x0 = __fmul2_rn(a, lo2(s[r])), x1 = __fmul2_rn(a, hi2(s[r]));
+        s[r] = make_float4(x0.x, x0.y, x1.x, x1.y);
+        p0 = __ffma2_rn(ka, x0, p0);
+        p1 = __ffma2_rn(ka, x1, p1);
+        if (out) {
+          const float2 qa = make_float2(sq[u][i], sq[u][i]);
+          r0 = __ffma2_rn(qa, x0, r0);
+          r1 = __ffma2_rn(qa, x1, r1);
+        }
+      }
+      red_p[par][ty][tx] = make_float4(p0.x, p0.y, p1.x, p1.y);
+      if (out) red_r[par][ty][tx] = make_float4(r0.x, r0.y, r1.x, r1.y);
+      __syncthreads();
+      float4 P = red_p[par][0][tx];
 #pragma unroll
       for (int y = 1; y < RP; ++y) {
-        const float4 c = red_r[y][tx];
-        R.x += c.x; R.y += c.y; R.z += c.z; R.w += c.w;
+        const float4 c = red_p[par][y][tx];
+        P.x += c.x; P.y += c.y; P.z += c.z; P.w += c.w;
       }
-      const float qk = s_qk;
-      TIn *ob = o + in_v + j0;
-      put(ob + 0, scale * (R.x + qk * u.x));
-      put(ob + 1, scale * (R.y + qk * u.y));
-      put(ob + 2, scale * (R.z + qk * u.z));
-      put(ob + 3, scale * (R.w + qk * u.w));
+      const int j0 = 4 * tx;
+      const float b = sb[u];
+      const float4 vj = *reinterpret_cast<const float4 *>(&sv[u][j0]);
+      const float4 uu = make_float4(b * (vj.x - P.x), b * (vj.y - P.y), b * (vj.z - P.z), b * (vj.w - P.w));
+      const float2 u0 = lo2(uu), u1 = hi2(uu);
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) {
+        const float2 ki = make_float2(sk[u][ty + r * RP], sk[u][ty + r * RP]);
+        const float2 x0 = __ffma2_rn(ki, u0, lo2(s[r])), x1 = __ffma2_rn(ki, u1, hi2(s[r]));
+        s[r] = make_float4(x0.x, x0.y, x1.x, x1.y);
+      }
+      if (t == nr - 1)  // the last accepted token: this state is committed
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) S4[(ty + r * RP) * TPR + tx] = s[r];
+      if (out && ty == 0) {
+        float4 R = red_r[par][0][tx];
+#pragma unroll
+        for (int y = 1; y < RP; ++y) {
+          const float4 c = red_r[par][y][tx];
+          R.x += c.x; R.y += c.y; R.z += c.z; R.w += c.w;
+        }
+        const float qk = sqk[u];
+        TIn *ob = o + ((size_t)bh * W + t) * DV + j0;
+        put(ob + 0, scale * (R.x + qk * uu.x));
+        put(ob + 1, scale * (R.y + qk * uu.y));
+        put(ob + 2, scale * (R.z + qk * uu.z));
+        put(ob + 3, scale * (R.w + qk * uu.w));
+      }
+      // red_*[par] is rewritten two tokens later, after the next token's barrier
     }
-    __syncthreads();  // this token's shared inputs and partial sums are consumed
   }
 }
 

@@ -5,10 +5,12 @@ tokens [r*T_r, (r+1)*T_r) of every chain.  A segment maps its entering state S
 to S~ + M S (the recurrence is linear in S), so
 
 1. every rank computes (S~_r, M_r) of its own segment: S~ is the final state of
-   a prefill from a zero state, M the final state of a prefill from h0 = I with
-   v = 0 (dk == dv);
-2. one exchange: all-gather of the pairs (2 x 64 KiB fp32 per chain per rank
-   at d = 128), NCCL over NVLink on a GPU group;
+   the segment run from a zero state, M = M_T ... M_1 the product of its token
+   transitions; on the tensor-core path one transition-only launch gives both
+   (no q loads, no outputs); elsewhere two prefills give them (S~ from a zero
+   state, M from h0 = I with v = 0, dk == dv);
+2. one exchange: one all-gather of each rank's packed pair [M | S~] (2 x 64 KiB
+   fp32 per chain at d = 128), NCCL over NVLink on a GPU group;
 3. rank R composes the state entering its segment from h0 and the pairs of
    ranks < R (kda_kcp_compose, on the device);
 4. rank R runs its prefill from that state: its outputs, and on the last rank
@@ -23,19 +25,36 @@ from __future__ import annotations
 from . import kda
 
 
+def pack(m, st):
+    """One flat buffer [M | S~] per rank (the payload of the single all-gather)."""
+    import torch
+    return torch.cat([m.reshape(-1), st.reshape(-1)])
+
+
+def unpack(flat, B, H, dk, dv):
+    n = B * H * dk * dk
+    return flat[:n].view(B, H, dk, dk), flat[n:n + B * H * dk * dv].view(B, H, dk, dv)
+
+
 class LibkdaOps:
     """The steps of KCP on the device, through libkda's C ABI."""
 
     @staticmethod
-    def transition(q, k, v, g, beta, scale=0.0):
+    def transition_packed(q, k, v, g, beta, scale=0.0):
+        """This rank's [M | S~] as one flat fp32 tensor."""
         import torch
         B, H, T, dk = q.shape
-        if v.shape[-1] != dk:
-            raise ValueError("cross-device KCP needs dk == dv (M is taken as the state from h0 = I)")
+        dv = v.shape[-1]
+        if q.dtype == torch.bfloat16 and dk == 128 and dv == 128:
+            flat = torch.empty(B * H * (dk * dk + dk * dv), dtype=torch.float32, device=q.device)
+            kda.chunk_transition(k, v, g, beta, out=flat)
+            return flat
+        if dv != dk:
+            raise ValueError("cross-device KCP on the CUDA-core path needs dk == dv (M is the state from h0 = I)")
         _, st = kda.chunk_fwd(q, k, v, g, beta, None, scale=scale)
         eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(B, H, dk, dk).contiguous()
         _, m = kda.chunk_fwd(q, k, torch.zeros_like(v), g, beta, eye, scale=scale)
-        return st, m
+        return pack(m, st)
 
     @staticmethod
     def compose(ms, sts, h0, like):
@@ -62,15 +81,16 @@ def kcp_prefill(q, k, v, g, beta, h0=None, *, group=None, scale=0.0, ops=LibkdaO
     state entering the whole sequence (the same on every rank, or None).
     Returns (o for this rank's tokens, state after this rank's segment): the
     last rank's state is the sequence's final state.  Every rank takes the
-    same collective steps (two all-gathers)."""
+    same collective step: one all-gather."""
     import torch
     import torch.distributed as dist
     rank, world = dist.get_rank(group), dist.get_world_size(group)
-    st, m = ops.transition(q, k, v, g, beta, scale)
-    st_all = [torch.empty_like(st) for _ in range(world)]
-    m_all = [torch.empty_like(m) for _ in range(world)]
-    dist.all_gather(st_all, st.contiguous(), group=group)
-    dist.all_gather(m_all, m.contiguous(), group=group)
-    like = st if h0 is None else h0
-    s_in = ops.compose(m_all[:rank], st_all[:rank], h0, like)
+    B, H, _, dk = q.shape
+    dv = v.shape[-1]
+    flat = ops.transition_packed(q, k, v, g, beta, scale).contiguous()
+    gathered = [torch.empty_like(flat) for _ in range(world)]
+    dist.all_gather(gathered, flat, group=group)
+    pairs = [unpack(gathered[r], B, H, dk, dv) for r in range(rank)]
+    like = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device) if h0 is None else h0
+    s_in = ops.compose([m for m, _ in pairs], [st for _, st in pairs], h0, like)
     return ops.prefill(q, k, v, g, beta, s_in, scale)

@@ -25,7 +25,8 @@ STATUS_NAMES = ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_SHAPE", "KDA_ERR_DTYPE
 EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
             "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate",
-            "kda_kcp_compose", "kda_spec_replay_verify"]
+            "kda_kcp_compose", "kda_spec_replay_verify", "kda_debug_set_wait_limit", "kda_debug_inject_stall",
+            "kda_chunk_fwd_outgate", "kda_chunk_transition"]
 
 
 class KdaError(RuntimeError):
@@ -64,6 +65,10 @@ def load_library():
             lib.kda_chunk_fwd_ckpt.restype = i
             lib.kda_chunk_fwd_gated.argtypes = [vp] * 5 + [f] + [vp] * 4 + [i] * 7 + [f, vp, sz, vp]
             lib.kda_chunk_fwd_gated.restype = i
+            lib.kda_chunk_fwd_outgate.argtypes = [vp] * 8 + [f, vp, vp] + [i] * 7 + [f, vp, sz, vp]
+            lib.kda_chunk_fwd_outgate.restype = i
+            lib.kda_chunk_transition.argtypes = [vp] * 6 + [i] * 6 + [vp]
+            lib.kda_chunk_transition.restype = i
             lib.kda_output_gate.argtypes = [vp, vp, vp, f, vp] + [i] * 5 + [vp]
             lib.kda_output_gate.restype = i
             lib.kda_kcp_compose.argtypes = [vp] * 4 + [i] * 5 + [vp]
@@ -76,6 +81,10 @@ def load_library():
             lib.kda_status_string.restype = ctypes.c_char_p
             lib.kda_get_device_status.argtypes = [vp]
             lib.kda_get_device_status.restype = i
+            lib.kda_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+            lib.kda_debug_set_wait_limit.restype = i
+            lib.kda_debug_inject_stall.argtypes = [i]
+            lib.kda_debug_inject_stall.restype = i
             lib.kda_version.argtypes = []
             lib.kda_version.restype = i
             lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 8 + [i] * 7 + [f, vp]
@@ -132,6 +141,19 @@ def kda_chunk_fwd_gated(q, k, v, z, A_log, g_min, beta, h0, o, h_T, B, H, T, dk,
                                               chunk_size, scale, workspace, workspace_bytes, stream)
 
 
+def kda_chunk_fwd_outgate(q, k, v, g, beta, h0, gate, rms_weight, eps, y, h_T, B, H, T, dk, dv, dtype, chunk_size,
+                          scale, workspace, workspace_bytes, stream) -> int:
+    """kda_chunk_fwd with the Eq. 6 output edge fused into the epilogue: writes
+    y = Sigmoid(gate) * RMSNorm_w(o) instead of o.  Returns the raw kda_status_t."""
+    return load_library().kda_chunk_fwd_outgate(q, k, v, g, beta, h0, gate, rms_weight, eps, y, h_T, B, H, T, dk, dv,
+                                                dtype, chunk_size, scale, workspace, workspace_bytes, stream)
+
+
+def kda_chunk_transition(k, v, g, beta, St, M, B, H, T, dk, dv, dtype, stream) -> int:
+    """Segment transition (S~, M) of every chain (Eq. 17).  Returns the raw kda_status_t."""
+    return load_library().kda_chunk_transition(k, v, g, beta, St, M, B, H, T, dk, dv, dtype, stream)
+
+
 def kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream) -> int:
     """Eq. 6 output edge: y = Sigmoid(gate) * RMSNorm(o).  Returns the raw kda_status_t."""
     return load_library().kda_output_gate(o, gate, rms_weight, eps, y, B, H, T, dv, dtype, stream)
@@ -165,6 +187,14 @@ def kda_recurrent_step(q, k, v, g, beta, S, o, B, H, dk, dv, dtype, scale, strea
 
 def kda_get_device_status(stream=None) -> int:
     return load_library().kda_get_device_status(stream)
+
+
+def kda_debug_set_wait_limit(ns: int) -> int:
+    return load_library().kda_debug_set_wait_limit(int(ns))
+
+
+def kda_debug_inject_stall(on: bool) -> int:
+    return load_library().kda_debug_inject_stall(1 if on else 0)
 
 
 # ---- torch helpers ---------------------------------------------------------
@@ -232,6 +262,53 @@ def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, h_T=None, scale=0.0, chunk_s
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
     return o, h_T
+
+
+def chunk_transition(k, v, g, beta, *, out=None, stream=None):
+    """(S~, M) of every chain's segment: S~ [B, H, dk, dv] and M [B, H, dk, dk]
+    fp32 (kda_chunk_transition).  `out`, if given, is one fp32 buffer of
+    B*H*(dk*dk + dk*dv) elements that receives M then S~ (so a rank can
+    publish both with one collective); the returned tensors are views of it."""
+    import torch
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    n = B * H
+    if out is None:
+        out = torch.empty(n * (dk * dk + dk * dv), dtype=torch.float32, device=k.device)
+    m = out[:n * dk * dk].view(B, H, dk, dk)
+    st = out[n * dk * dk:n * (dk * dk + dk * dv)].view(B, H, dk, dv)
+    code = kda_chunk_transition(_ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(st), _ptr(m), B, H, T, dk, dv,
+                                _dtype_code(k), _stream(stream))
+    if code != KDA_OK:
+        raise KdaError(code, "kda_chunk_transition")
+    return st, m
+
+
+def chunk_fwd_outgate(q, k, v, g, beta, gate, rms_weight, h0=None, *, eps=1e-6, y=None, h_T=None, scale=0.0,
+                      chunk_size=0, output_final_state=True, workspace=None, stream=None):
+    """Prefill with the fused Eq. 6 output edge: gate [B, H, T, dv] (dtype of q),
+    rms_weight [H, dv] fp32.  Allocates y / h_T / workspace when not given.
+    Returns (y, h_T)."""
+    import torch
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if y is None:
+        y = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_T is None and output_final_state:
+        h_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    ws = kda_chunk_fwd_workspace_size(B, H, T, dk, dv, dt, chunk_size)
+    if ws == (1 << 64) - 1:
+        raise KdaError(2, "kda_chunk_fwd_workspace_size")
+    if ws > 0 and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = kda_chunk_fwd_outgate(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(gate), _ptr(rms_weight),
+                               float(eps), _ptr(y), _ptr(h_T), B, H, T, dk, dv, dt, chunk_size, float(scale),
+                               _ptr(workspace), wbytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_outgate")
+    return y, h_T
 
 
 def chunk_fwd_gated(q, k, v, z, A_log, beta, h0=None, *, g_min=-5.0, o=None, h_T=None, scale=0.0, chunk_size=0,

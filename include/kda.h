@@ -207,15 +207,57 @@ kda_status_t kda_output_gate(const void *o, const void *gate, const float *rms_w
                              int B, int H, int T, int dv, kda_dtype_t dtype, kda_stream_t stream);
 
 /*
+ * Prefill with the output edge of the KDA layer fused into the output
+ * epilogue (Kimi K3 report, section 2.1.1, Eq. 6, without its projections):
+ *     y_t = Sigmoid(gate_t) * w_h * o_t / sqrt(mean_j(o_t[j]^2) + eps),
+ * o_t being what kda_chunk_fwd would write (the RMS is per token and head,
+ * over dv).  On the tensor-core path the epilogue normalises and gates each
+ * output tile on chip, so o never reaches memory; on the CUDA-core path the
+ * prefill writes o into y's buffer and the edge runs in place after it.
+ * Arguments as for kda_chunk_fwd, with o replaced by
+ *   gate       : [B, H, T, dv] in dtype (W_g x split into heads), 16-byte aligned
+ *   rms_weight : [H, dv] fp32, 16-byte aligned;   eps >= 0
+ *   y          : [B, H, T, dv] in dtype, written; must not overlap any input
+ *                (gate and rms_weight included)
+ * Same workspace size as kda_chunk_fwd.  Errors as for kda_chunk_fwd.
+ */
+kda_status_t kda_chunk_fwd_outgate(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                                   const float *h0, const void *gate, const float *rms_weight, float eps, void *y,
+                                   float *h_T, int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                   int chunk_size, float scale, void *workspace, size_t workspace_bytes,
+                                   kda_stream_t stream);
+
+/*
+ * Segment transition of KDA context parallelism (Kimi K3 report, section
+ * 5.1.2, Eq. 17).  The recurrence is linear in its entering state: a prefill
+ * of these T tokens that starts from S ends in  S~ + M S,  with
+ *     M = M_T ... M_1,   M_t = (I - beta_t k_t k_t^T) Diag(alpha_t),
+ * and S~ the end state from S = 0.  This call computes both for every chain in
+ * one launch, without q and without writing any output (the transition-only
+ * form of the tensor-core kernel: two CTAs per chain, one carrying S~ from
+ * zero, one carrying M from I with no value write), so a rank can publish its
+ * pair before it knows its entering state.
+ *   k, g : [B, H, T, dk]; v : [B, H, T, dv]; beta : [B, H, T]   (dtype)
+ *   St   : [B, H, dk, dv] fp32, written (S~)
+ *   M    : [B, H, dk, dk] fp32, written, row-major (M[i][j] multiplies S's row j)
+ * bf16 with dk = dv = 128 only (KDA_ERR_DTYPE / KDA_ERR_SHAPE otherwise).
+ * T = 0 gives S~ = 0 and M = I.  k, v, g, St, M 16-byte aligned; St and M must
+ * not overlap each other or the inputs.  Allocates nothing.
+ */
+kda_status_t kda_chunk_transition(const void *k, const void *v, const void *g, const void *beta, float *St,
+                                  float *M, int B, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                                  kda_stream_t stream);
+
+/*
  * Cross-device KDA context parallelism, prefix step (Kimi K3 report, section
  * 5.1.2, Eq. 17).  Each rank holds one segment of every chain; a segment maps
  * its entering state S to S~ + M S.  After one all-gather of the (M_r, S~_r)
  * pairs (the caller's NCCL collective), rank R composes the state entering its
  * segment,
  *     S_in = M_{R-1} (... (M_0 h0 + S~_0) ...) + S~_{R-1},
- * and runs its prefill from S_in.  (M_r, S~_r) of a segment come from two
- * prefill calls on it: S~ = h_T from a zero state, M = h_T from h0 = I with
- * v = 0 (dk == dv).
+ * and runs its prefill from S_in.  (M_r, S~_r) of a segment come from
+ * kda_chunk_transition (or, on the CUDA-core path, from two prefill calls on
+ * it: S~ = h_T from a zero state, M = h_T from h0 = I with v = 0, dk == dv).
  *   M    : [R, B, H, dk, dk] fp32;  St : [R, B, H, dk, dv] fp32 (rank-major)
  *   h0   : [B, H, dk, dv] fp32, or NULL for a zero initial state
  *   S_in : [B, H, dk, dv] fp32, written; must not overlap the inputs
@@ -289,6 +331,25 @@ const char *kda_status_string(kda_status_t s);
  * recorded, KDA_ERR_CUDA if synchronising failed.
  */
 kda_status_t kda_get_device_status(kda_stream_t stream);
+
+/*
+ * Failure-detection testing aids (host-side fault injection; never needed in
+ * production).  The tensor-core prefill kernel's cross-role waits are bounded:
+ * a wait that does not complete within the limit aborts the CTA (no further
+ * tensor-core work, every issued copy and MMA drained before its tensor memory
+ * is released), records KDA_ERR_TIMEOUT in the device status word and returns,
+ * so the context stays usable; the outputs of that call are then undefined.
+ *
+ * kda_debug_set_wait_limit: wall-time limit of those waits for calls enqueued
+ *   afterwards, in nanoseconds (0 restores the default of 2 s).  Process-wide.
+ * kda_debug_inject_stall: when on, prefill calls on the tensor-core path
+ *   enqueued afterwards first wait on a barrier nothing ever arrives on, so
+ *   the wait runs out after the limit above and the call aborts as described.
+ *   Process-wide; turn it off again to resume normal operation.
+ * Both return KDA_OK.
+ */
+kda_status_t kda_debug_set_wait_limit(unsigned long long ns);
+kda_status_t kda_debug_inject_stall(int on);
 
 /* Library version, e.g. 100 for 0.1.0. */
 int kda_version(void);

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from gated_delta_rule_117_b200 import kda, synth
-from gated_delta_rule_117_b200.kcp import LibkdaOps
+from gated_delta_rule_117_b200.kcp import LibkdaOps, unpack
 from parity_util import TOL, oracle_prefill, rel_l2, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -17,10 +17,13 @@ pytestmark = pytest.mark.gpu
 def _emulate(d, R, T):
     n = T // R
     seg = lambda r: [d[k][:, :, r * n:(r + 1) * n].contiguous() for k in ("q", "k", "v", "g", "beta")]
-    pairs = [LibkdaOps.transition(*seg(r)) for r in range(R)]  # every rank's (S~, M)
+    B, H, _, dk = d["q"].shape
+    dv = d["v"].shape[-1]
+    # every rank's packed [M | S~] (what the all-gather exchanges)
+    pairs = [unpack(LibkdaOps.transition_packed(*seg(r)), B, H, dk, dv) for r in range(R)]
     outs, hT = [], None
     for r in range(R):  # rank r after the all-gather
-        s_in = LibkdaOps.compose([m for _, m in pairs[:r]], [st for st, _ in pairs[:r]], d["h0"], d["h0"])
+        s_in = LibkdaOps.compose([m for m, _ in pairs[:r]], [st for _, st in pairs[:r]], d["h0"], d["h0"])
         o, hT = LibkdaOps.prefill(*seg(r), s_in)
         outs.append(o)
     return torch.cat(outs, dim=2), hT
@@ -64,3 +67,24 @@ def test_compose_matches_fp64():
     assert kda.kda_kcp_compose(None, None, hd.data_ptr(), out.data_ptr(), 0, B, H, dk, dv, None) == 0
     torch.cuda.synchronize()
     assert torch.equal(out, hd)
+
+
+@pytest.mark.parametrize("T", [0, 1, 45, 300])
+def test_transition_entry_point_matches_oracle(T):
+    # kda_chunk_transition: S~ (state from zero) and M = M_T ... M_1 (Eq. 17) in one launch
+    import oracle
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=2, H=2, T=T, seed=80 + T)
+    x = synth.prefill_inputs(w)
+    d = to_dev(x)
+    st, m = kda.chunk_transition(d["k"], d["v"], d["g"], d["beta"])
+    assert kda.kda_get_device_status() == 0
+    f = lambda t: t.double().numpy()
+    for b in range(2):
+        for h in range(2):
+            if T == 0:
+                assert torch.equal(m[b, h].cpu(), torch.eye(128)) and torch.count_nonzero(st[b, h]) == 0
+                continue
+            M_ref = oracle.transition(f(x["k"][b, h]), f(x["g"][b, h]), f(x["beta"][b, h]))
+            _, S_ref = oracle.recurrent(f(x["q"][b, h]), f(x["k"][b, h]), f(x["v"][b, h]), f(x["g"][b, h]),
+                                        f(x["beta"][b, h]))
+            assert rel_l2(m[b, h], M_ref) <= TOL["bf16"] and rel_l2(st[b, h], S_ref) <= TOL["bf16"]

@@ -62,15 +62,16 @@ class _OracleOps:
     device kernels): the orchestration, not the arithmetic, is under test."""
 
     @staticmethod
-    def transition(q, k, v, g, beta, scale=0.0):
+    def transition_packed(q, k, v, g, beta, scale=0.0):
         import numpy as np
         import oracle
+        from gated_delta_rule_117_b200 import kcp
         a = [t.double().numpy() for t in (q, k, v, g, beta)]
         _, st = oracle.recurrent(*a)
-        dk = q.shape[-1]
-        eye = np.broadcast_to(np.eye(dk), q.shape[:2] + (dk, dk)).copy()
-        _, m = oracle.recurrent(a[0], a[1], np.zeros_like(a[2]), a[3], a[4], eye)
-        return torch.from_numpy(st), torch.from_numpy(m)
+        B, H = q.shape[:2]
+        m = np.stack([np.stack([oracle.transition(a[1][b, h], a[3][b, h], a[4][b, h]) for h in range(H)])
+                      for b in range(B)])
+        return kcp.pack(torch.from_numpy(m), torch.from_numpy(st))
 
     @staticmethod
     def compose(ms, sts, h0, like):
@@ -96,7 +97,14 @@ def _kcp_worker(rank, world, port, out):
         x = synth.prefill_inputs(w)
         n = w.T // world
         sl = {k2: (x[k2][:, :, rank * n:(rank + 1) * n] if k2 != "h0" else x[k2]) for k2 in x}
-        o, hT = kcp.kcp_prefill(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], x["h0"], ops=_OracleOps)
+        calls = []
+        real = dist.all_gather
+        dist.all_gather = lambda *a, **kw: (calls.append(1), real(*a, **kw))[1]
+        try:
+            o, hT = kcp.kcp_prefill(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], x["h0"], ops=_OracleOps)
+        finally:
+            dist.all_gather = real
+        assert len(calls) == 1  # one exchange of the packed (M, S~) pairs
         out[rank] = (o.numpy(), hT.numpy())
         dist.barrier()
     finally:
