@@ -69,12 +69,17 @@ def test_compose_matches_fp64():
     assert torch.equal(out, hd)
 
 
-@pytest.mark.parametrize("T", [0, 1, 45, 300])
-def test_transition_entry_point_matches_oracle(T):
-    # kda_chunk_transition: S~ (state from zero) and M = M_T ... M_1 (Eq. 17) in one launch
+@pytest.mark.parametrize("T,g_scale", [(0, 1.0), (1, 1.0), (45, 1.0), (45, 0.05), (300, 0.01)])
+def test_transition_entry_point_matches_oracle(T, g_scale):
+    # kda_chunk_transition: S~ (state from zero) and M = M_T ... M_1 (Eq. 17) in one launch.
+    # At the workloads' decay (g ~ -2.5 per token) M falls below fp32's normal range
+    # within ~35 tokens (e^-87), where relative error means nothing: there M is
+    # checked in absolute terms; the scaled-down decays keep M representable and
+    # check it in relative L2.
     import oracle
     w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=2, H=2, T=T, seed=80 + T)
     x = synth.prefill_inputs(w)
+    x["g"] = (x["g"].float() * g_scale).to(x["g"].dtype)
     d = to_dev(x)
     st, m = kda.chunk_transition(d["k"], d["v"], d["g"], d["beta"])
     assert kda.kda_get_device_status() == 0
@@ -87,4 +92,8 @@ def test_transition_entry_point_matches_oracle(T):
             M_ref = oracle.transition(f(x["k"][b, h]), f(x["g"][b, h]), f(x["beta"][b, h]))
             _, S_ref = oracle.recurrent(f(x["q"][b, h]), f(x["k"][b, h]), f(x["v"][b, h]), f(x["g"][b, h]),
                                         f(x["beta"][b, h]))
-            assert rel_l2(m[b, h], M_ref) <= TOL["bf16"] and rel_l2(st[b, h], S_ref) <= TOL["bf16"]
+            assert rel_l2(st[b, h], S_ref) <= TOL["bf16"]
+            if np.abs(M_ref).max() > 1e-30:
+                assert rel_l2(m[b, h], M_ref) <= TOL["bf16"]
+            else:
+                assert np.abs(m[b, h].double().cpu().numpy() - M_ref).max() <= 1e-30
