@@ -43,7 +43,11 @@
 //                        rescaled operands and the Gram MMAs (chunk t + 2);
 //   warps 8-11  token B: A, L, the triangular solve, the U/W~ MMAs and -W~
 //                        (chunk t + 1).
-// One elected lane of a converged warp issues each MMA and TMA copy.  The
+// One elected lane of a converged warp issues each MMA and TMA copy.  The issue
+// loops stay rolled: in isolation an unrolled loop issues a tcgen05.mma in ~20
+// cycles against ~70, but inside this pipeline the MMAs queue behind the other
+// roles' tensor work either way, and the larger code slowed every other stage
+// (three warpgroups share each sub-partition's instruction cache).  The
 // groups hand chunks over through mbarrier rings indexed by chunk parity;
 // the buffers a later stage reads are double buffered (the per-channel decay
 // factors, which the chain reads last, triple buffered).  The chain hands a
@@ -69,6 +73,7 @@ constexpr int D = 128;    // dk = dv
 constexpr int NT = 384;   // 12 warps: chain warpgroup + two token warpgroups
 constexpr uint32_t kWaitLimit = 1u << 22;  // polls; seconds, far beyond any real wait
 constexpr uint32_t kBarChain = 1, kBarTokA = 2, kBarTokB = 3;
+constexpr int kFinishedEarly = 2;  // abort-flag value of a run that stopped early without an error
 
 // ---- shared memory (byte offsets from a 1024-aligned base) -------------------
 // "h0/h1" = channel blocks 0..63 / 64..127 of a [tokens x 128] bf16 tile stored
@@ -558,6 +563,7 @@ __global__ void __launch_bounds__(NT, 1)
       // two chunks behind, so the buffers of parity pb may take chunk t + 2
       mma_commit_warp(&x.bar[B_CD0 + pb]);
     };
+    bool finished = false;  // the M run stopped early on a vanished state (see below)
     // fused Eq. 6 edge: this thread's RMSNorm weight; the gate tile of chunk 0
     float wgt = 0.f;
     int gate_issued = -1;  // last chunk whose gate tile was requested (abort path)
@@ -681,6 +687,22 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (has_next) fence_proxy_async_smem();
       }
+      // Exact early finish of the M run (transition from I with v = 0): its
+      // update is homogeneous, so once the carried state is exactly zero every
+      // later chunk leaves it exactly zero (zero operands give zero products):
+      // the run stops, like an abort but without an error, and stores those
+      // zeros -- the result this kernel would have computed over the rest of
+      // the segment, bit for bit.  Under decaying gates the state vanishes
+      // within a few chunks; a state that does not vanish runs to the end.
+      if (kTrans && v_zero && has_next) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int i = 0; i < D / 2; ++i) bits |= (__float_as_uint(S[i].x) | __float_as_uint(S[i].y)) & 0x7fffffffu;
+        if (named_sync_and(kBarChain, 128, bits == 0u)) {
+          finished = true;
+          if (e == 0) *x.abort = kFinishedEarly;
+        }
+      }
       tc_fence_before();
       const bool go = named_sync_and(kBarChain, 128, *x.abort == 0);
       // [O | V~](t+1) is issued as soon as token B has finished chunk t + 1;
@@ -775,12 +797,13 @@ __global__ void __launch_bounds__(NT, 1)
     if (kOut && warp == 0 && lane == 0 && *x.abort && gate_issued >= 0)  // let the last gate copy land
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_GATE], (uint32_t)gate_issued & 1u); ++i) {
       }
-    if (*x.abort == 0 && hdst && kind == 2 && !p.m_rowmajor) {
+    const bool valid = *x.abort == 0 || finished;
+    if (valid && hdst && kind == 2 && !p.m_rowmajor) {
       // the segment transition is stored transposed (row e = column e of M) for the scan
       float4 *row = reinterpret_cast<float4 *>(hdst + (size_t)e * D);
 #pragma unroll
       for (int i = 0; i < D / 4; ++i) row[i] = make_float4(S[2 * i].x, S[2 * i].y, S[2 * i + 1].x, S[2 * i + 1].y);
-    } else if (*x.abort == 0 && hdst) {
+    } else if (valid && hdst) {
 #pragma unroll
       for (int i = 0; i < D / 2; ++i) {
         hdst[(2 * i) * D + e] = S[i].x;

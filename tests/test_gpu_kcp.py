@@ -97,3 +97,24 @@ def test_transition_entry_point_matches_oracle(T, g_scale):
                 assert rel_l2(m[b, h], M_ref) <= TOL["bf16"]
             else:
                 assert np.abs(m[b, h].double().cpu().numpy() - M_ref).max() <= 1e-30
+
+
+def test_transition_of_a_vanishing_segment_finishes_early_and_exactly():
+    # At the workloads' decay the M run's state underflows to exactly zero within a
+    # few chunks; from then on every chunk keeps it exactly zero, so the kernel
+    # stops that run early and stores the zeros (no error recorded).  S~ still
+    # runs to the end and must match the oracle.
+    import oracle
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=2, T=4000, seed=91)
+    x = synth.prefill_inputs(w)
+    d = to_dev(x)
+    st, m = kda.chunk_transition(d["k"], d["v"], d["g"], d["beta"])
+    assert kda.kda_get_device_status() == 0
+    assert torch.count_nonzero(m) == 0
+    f = lambda t: t.double().numpy()
+    for h in range(2):
+        M_ref = oracle.transition(f(x["k"][0, h]), f(x["g"][0, h]), f(x["beta"][0, h]))
+        assert np.abs(M_ref).max() < 1e-30
+        _, S_ref = oracle.recurrent(f(x["q"][0, h]), f(x["k"][0, h]), f(x["v"][0, h]), f(x["g"][0, h]),
+                                    f(x["beta"][0, h]))
+        assert rel_l2(st[0, h], S_ref) <= TOL["bf16"]
