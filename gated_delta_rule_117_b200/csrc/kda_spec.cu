@@ -17,7 +17,8 @@
 // staged in shared memory once (in blocks of WB tokens) while the state load
 // is in flight; the column partial sums are double-buffered by token parity,
 // so each token costs one barrier; the q-side sums are formed only for the
-// tokens whose output is verified.
+// tokens whose output is verified.  For dk = dv = 128 a warp-sliced variant
+// (below) replaces the per-token barrier with shuffles inside each warp.
 #include <cuda_bf16.h>
 
 #include "kda_internal.cuh"
@@ -148,6 +149,116 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
   }
 }
 
+// dk = dv = 128: a warp owns a 16-column slice of the state over all 128 rows
+// (lane = row group rg = lane / 4 of 8, column group cg = lane % 4 of 4 float4
+// columns; rows rg, rg + 8, ..., rg + 120 in registers), so the column sums
+// over dk finish with three butterfly shuffles inside the warp and a token
+// needs no barrier: the warps of a CTA run through the window independently.
+constexpr int kD = 128, kWarps = 8, kRowsPT = 16, kWB = 8;
+
+template <typename TIn>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+    spec_replay_verify_d128_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
+                                   const TIn *__restrict__ v, const TIn *__restrict__ g,
+                                   const TIn *__restrict__ beta, float *S, TIn *__restrict__ o,
+                                   const int *__restrict__ n_replay, int H, int W, float scale) {
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rg = lane >> 2, cg = lane & 3;
+  const int col4 = 4 * warp + cg;  // float4 column index of this thread (columns 4*col4 .. +3)
+  // staged window block: per token and row {alpha, k} and q; v; beta; q.k
+  __shared__ float2 sak[kWB][kD];
+  __shared__ float sq[kWB][kD], sv[kWB][kD], sb[kWB], sqk[kWB];
+
+  const int nr = min(max(n_replay[bh / H], 0), W);
+  float4 *S4 = reinterpret_cast<float4 *>(S + (size_t)bh * kD * kD);
+  float4 s[kRowsPT];
+#pragma unroll
+  for (int r = 0; r < kRowsPT; ++r) s[r] = S4[(rg + 8 * r) * (kD / 4) + col4];  // in flight while staging
+
+  for (int t0 = 0; t0 < W; t0 += kWB) {
+    const int nb = min(kWB, W - t0);
+    if (t0 > 0) __syncthreads();  // every warp is done with the previous block
+    for (int e = tid; e < nb * kD; e += kWarps * 32) {
+      const int u = e / kD, i = e % kD;
+      const size_t in = ((size_t)bh * W + t0 + u) * kD + i;
+      sak[u][i] = make_float2(expf(to_f(g[in])), to_f(k[in]));
+      sq[u][i] = to_f(q[in]);
+      sv[u][i] = to_f(v[in]);
+    }
+    if (tid < nb) sb[tid] = to_f(beta[(size_t)bh * W + t0 + tid]);
+    __syncthreads();
+    if (warp < nb) {  // q . k of token `warp`
+      float acc = 0.f;
+#pragma unroll
+      for (int i = lane; i < kD; i += 32) acc += sq[warp][i] * sak[warp][i].y;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) sqk[warp] = acc;
+    }
+    __syncthreads();
+    for (int u = 0; u < nb; ++u) {
+      const int t = t0 + u;
+      const bool out = t >= nr;  // bonus / draft token: its output is verified
+      float2 p0 = make_float2(0.f, 0.f), p1 = p0, r0 = p0, r1 = p0;
+#pragma unroll
+      for (int r = 0; r < kRowsPT; ++r) {
+        const float2 ak = sak[u][rg + 8 * r];
+        const float2 a = make_float2(ak.x, ak.x), ka = make_float2(ak.y, ak.y);
+        const float2 x0 = __fmul2_rn(a, lo2(s[r])), x1 = __fmul2_rn(a, hi2(s[r]));
+        s[r] = make_float4(x0.x, x0.y, x1.x, x1.y);
+        p0 = __ffma2_rn(ka, x0, p0);
+        p1 = __ffma2_rn(ka, x1, p1);
+        if (out) {
+          const float qi = sq[u][rg + 8 * r];
+          const float2 qa = make_float2(qi, qi);
+          r0 = __ffma2_rn(qa, x0, r0);
+          r1 = __ffma2_rn(qa, x1, r1);
+        }
+      }
+      // column sums over the 8 row groups (lane bits 2-4): butterfly, every lane gets the total
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        p0.x += __shfl_xor_sync(0xffffffffu, p0.x, off);
+        p0.y += __shfl_xor_sync(0xffffffffu, p0.y, off);
+        p1.x += __shfl_xor_sync(0xffffffffu, p1.x, off);
+        p1.y += __shfl_xor_sync(0xffffffffu, p1.y, off);
+        if (out) {
+          r0.x += __shfl_xor_sync(0xffffffffu, r0.x, off);
+          r0.y += __shfl_xor_sync(0xffffffffu, r0.y, off);
+          r1.x += __shfl_xor_sync(0xffffffffu, r1.x, off);
+          r1.y += __shfl_xor_sync(0xffffffffu, r1.y, off);
+        }
+      }
+      const float b = sb[u];
+      const float4 vj = *reinterpret_cast<const float4 *>(&sv[u][4 * col4]);
+      const float2 u0 = make_float2(b * (vj.x - p0.x), b * (vj.y - p0.y));
+      const float2 u1 = make_float2(b * (vj.z - p1.x), b * (vj.w - p1.y));
+      // the state after the window's last token is neither committed nor read
+      // by any output (o needs only r and u), unless that token is replayed
+      if (t + 1 < W || t == nr - 1) {
+#pragma unroll
+        for (int r = 0; r < kRowsPT; ++r) {
+          const float ki1 = sak[u][rg + 8 * r].y;
+          const float2 ki = make_float2(ki1, ki1);
+          const float2 x0 = __ffma2_rn(ki, u0, lo2(s[r])), x1 = __ffma2_rn(ki, u1, hi2(s[r]));
+          s[r] = make_float4(x0.x, x0.y, x1.x, x1.y);
+        }
+      }
+      if (t == nr - 1)  // the last accepted token: this state is committed
+#pragma unroll
+        for (int r = 0; r < kRowsPT; ++r) S4[(rg + 8 * r) * (kD / 4) + col4] = s[r];
+      if (out && rg == 0) {
+        const float qk = sqk[u];
+        TIn *ob = o + ((size_t)bh * W + t) * kD + 4 * col4;
+        put(ob + 0, scale * (r0.x + qk * u0.x));
+        put(ob + 1, scale * (r0.y + qk * u0.y));
+        put(ob + 2, scale * (r1.x + qk * u1.x));
+        put(ob + 3, scale * (r1.y + qk * u1.y));
+      }
+    }
+  }
+}
+
 template <int DK, int DV, typename TIn>
 cudaError_t launch_t(const SpecArgs &a, cudaStream_t st) {
   spec_replay_verify_kernel<DK, DV, TIn><<<a.B * a.H, SpecShape<DK, DV>::NT, 0, st>>>(
@@ -158,6 +269,12 @@ cudaError_t launch_t(const SpecArgs &a, cudaStream_t st) {
 
 template <typename TIn>
 cudaError_t launch_dt(const SpecArgs &a, cudaStream_t st) {
+  if (a.dk == kD && a.dv == kD) {
+    spec_replay_verify_d128_kernel<TIn><<<a.B * a.H, kWarps * 32, 0, st>>>(
+        (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
+        (TIn *)a.o, a.n_replay, a.H, a.W, a.scale);
+    return cudaGetLastError();
+  }
 #define KDA_SP_CASE(DKv, DVv) \
   if (a.dk == DKv && a.dv == DVv) return launch_t<DKv, DVv, TIn>(a, st);
 #define KDA_SP_ROW(DKv) KDA_SP_CASE(DKv, 16) KDA_SP_CASE(DKv, 32) KDA_SP_CASE(DKv, 64) KDA_SP_CASE(DKv, 128)
