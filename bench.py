@@ -328,7 +328,16 @@ def time_prefill(args, w, d, plan, kda, torch, flush, dev, clk=None, dist=None):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    check_device_status(kda, "kda_chunk_fwd")
     return [a.elapsed_time(b) for a, b in ev], o, hT
+
+
+def check_device_status(kda, what):
+    """A timed run whose kernels recorded an error (a bounded wait that gave up)
+    is not a measurement: raise instead of reporting its time."""
+    st = kda.kda_get_device_status(None)
+    if st != 0:
+        raise kda.KdaError(st, what + " (device status after the timed steps)")
 
 
 def prefill_figures(w, plan, ms, pk, pk_kind, synth):
@@ -575,6 +584,7 @@ def measure_ckpt(args, w, d, h0, o, hT, ws, flush, kda, torch, plain_ms):
         step()
         b.record()
     torch.cuda.synchronize()
+    check_device_status(kda, "kda_chunk_fwd_ckpt")
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
     return {"interval": CKPT_INTERVAL, "checkpoints_per_chain": n, "ms_per_step": ms,
@@ -611,6 +621,7 @@ def measure_gate(args, w, d, h0, o, hT, ws, flush, synth, kda, torch, plain_ms):
         step()
         b.record()
     torch.cuda.synchronize()
+    check_device_status(kda, "kda_chunk_fwd_gated")
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
     e = 2 if w.dtype == "bf16" else 4
@@ -649,6 +660,7 @@ def measure_outgate_fused(args, w, d, h0, hT, ws, flush, kda, torch, plain_ms, s
         step()
         b.record()
     torch.cuda.synchronize()
+    check_device_status(kda, "kda_chunk_fwd_outgate")
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     e = 2 if w.dtype == "bf16" else 4
     launches = kda.kda_chunk_fwd_plan(B, H, T, dk, dv, dt, args.chunk_size)["launches"]
@@ -751,6 +763,7 @@ def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
             step()
         b.record(stream)
         torch.cuda.synchronize()
+        check_device_status(kda, "kda_chunk_fwd (e2e)")
         ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist, dev)
     finally:
         for n, (t, reg) in pinned.items():

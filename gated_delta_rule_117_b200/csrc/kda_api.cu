@@ -404,10 +404,53 @@ kda_status_t kda_kcp_compose(const float *M, const float *St, const float *h0, f
              : KDA_ERR_CUDA;
 }
 
+namespace {
+kda_status_t spec_replay(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
+                         void *o, const int *n_replay, int B, int H, int W, int dk, int dv, kda_dtype_t dtype,
+                         float scale, const float *A_log, float g_min, const void *gate, const float *rms_w, float eps,
+                         kda_stream_t stream);
+}  // namespace
+
+kda_status_t kda_spec_replay_verify_fused(const void *q, const void *k, const void *v, const void *z,
+                                          const float *A_log, float g_min, const void *beta, float *S,
+                                          const void *gate, const float *rms_weight, float eps, void *y,
+                                          const int *n_replay, int B, int H, int W, int dk, int dv,
+                                          kda_dtype_t dtype, float scale, kda_stream_t stream) {
+  if (B < 0 || H < 0 || W < 0) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
+  if (dk != 128 || dv != 128) return KDA_ERR_SHAPE;
+  if (!(g_min >= -5.f && g_min < 0.f)) return KDA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!(eps >= 0.f) || !isfinite(eps)) return KDA_ERR_INVALID_ARG;
+  if (B * H == 0 || W == 0) return KDA_OK;
+  if (!A_log || !gate || !rms_weight) return KDA_ERR_INVALID_ARG;
+  if (((uintptr_t)A_log & 3u) || ((uintptr_t)rms_weight & 3u)) return KDA_ERR_ALIGNMENT;
+  const size_t e = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+  if ((uintptr_t)gate % e) return KDA_ERR_ALIGNMENT;
+  const size_t n = (size_t)B * H;
+  const Range ry = range_of(y, n * W * dv * e), rg = range_of(gate, n * W * dv * e),
+              ra = range_of(A_log, (size_t)H * dk * 4), rw = range_of(rms_weight, (size_t)H * dv * 4),
+              rS = range_of(S, n * dk * dv * 4);
+  if (overlap(ry, rg) || overlap(ry, ra) || overlap(ry, rw) || overlap(rS, rg) || overlap(rS, ra) || overlap(rS, rw))
+    return KDA_ERR_ALIAS;
+  return spec_replay(q, k, v, z, beta, S, y, n_replay, B, H, W, dk, dv, dtype, scale, A_log, g_min, gate, rms_weight,
+                     eps, stream);
+}
+
 kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v, const void *g,
                                     const void *beta, float *S, void *o, const int *n_replay, int B,
                                     int H, int W, int dk, int dv, kda_dtype_t dtype, float scale,
                                     kda_stream_t stream) {
+  return spec_replay(q, k, v, g, beta, S, o, n_replay, B, H, W, dk, dv, dtype, scale, nullptr, 0.f, nullptr, nullptr,
+                     0.f, stream);
+}
+
+}  // extern "C"
+
+namespace {
+kda_status_t spec_replay(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
+                         void *o, const int *n_replay, int B, int H, int W, int dk, int dv, kda_dtype_t dtype,
+                         float scale, const float *A_log, float g_min, const void *gate, const float *rms_w, float eps,
+                         kda_stream_t stream) {
   if (B < 0 || H < 0 || W < 0) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_DTYPE;
   if (!supported_d(dk) || !supported_d(dv)) return KDA_ERR_SHAPE;
@@ -435,8 +478,16 @@ kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v,
   a.B = B; a.H = H; a.W = W; a.dk = dk; a.dv = dv;
   a.bf16 = dtype == KDA_DTYPE_BF16;
   a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
+  a.A_log = A_log;
+  a.g_min = g_min;
+  a.gate = gate;
+  a.rms_w = rms_w;
+  a.eps = eps;
   return kda::launch_spec_replay_verify(a, (cudaStream_t)stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
+}  // namespace
+
+extern "C" {
 
 kda_status_t kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
                                 const void *beta, float *S, void *o, int B, int H, int dk, int dv,

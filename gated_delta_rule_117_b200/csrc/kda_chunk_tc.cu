@@ -137,6 +137,8 @@ enum {
   B_CD1,
   B_DRAIN,     // every MMA issued by the three issuing warps is done (count 3; before TMEM is released)
   B_GATE,      // the output-gate tile of the chunk landed (fused Eq. 6 edge; TMA)
+  B_OUT0,      // [2] the chain's dS / O MMAs of the chunk are done: token B may write its output tile
+  B_OUT1,
   B_NEVER,     // nothing arrives here: the wait of an injected stall (failure-detection tests)
   B_COUNT
 };
@@ -489,6 +491,7 @@ __global__ void __launch_bounds__(NT, 1)
   const int nchunks = (te - tb + C - 1) / C;
   const bool v_zero = kTrans && kind == 2;
   const bool store_o = !kTrans;
+  constexpr bool out_b = !kTrans && !kOut;  // token B writes the plain output tiles
   const float *h0src = nullptr;
   float *hdst = nullptr;
   if (p.mode == kModeChain) {
@@ -635,6 +638,9 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
         mma_commit_warp(&x.bar[B_DS]);
+        // a second tracker of the same MMAs, indexed by chunk parity: token B waits on it
+        // two chunks later, when B_DS may already have completed again (same parity)
+        if (out_b) mma_commit_warp(&x.bar[B_OUT0 + pb]);
       }
       // the next chunk's e^rho (written by token A) is needed to form S~^T(t+1)
       if (has_next) wait_bar(x, B_DEC0 + (pb ^ 1), (uint32_t)((t + 1) >> 1) & 1u);
@@ -713,12 +719,13 @@ __global__ void __launch_bounds__(NT, 1)
         issue_v1(t + 1);
         issued = true;
       }
-      // output tile of chunk t (its TMEM half is not touched by chunk t + 1):
-      // column e goes into a swizzled shared tile that one TMA store writes out
-      // (rows past the end of the sequence are clipped by the tensor map)
-      if (store_o) {
+      // output tile of chunk t with the fused Eq. 6 edge (the plain output tile is
+      // written by token B, off the chain): column e goes into a swizzled shared
+      // tile that one TMA store writes out (rows past the end of the sequence are
+      // clipped by the tensor map)
+      if (store_o && kOut) {
         unsigned char *ot = sm + kOst + (e >> 6) * 4096;
-        if (kOut) {
+        {
           // Eq. 6 edge: y[r][e] = Sigmoid(gate[r][e]) w[e] o[r][e] / rms(o[r]), the rms
           // over the 128 channels, i.e. across the four chain warps
           float ov[32], v[32];
@@ -763,16 +770,6 @@ __global__ void __launch_bounds__(NT, 1)
               *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(r, e & 63)) = __float2bfloat16_rn(ov[r] * rr[u] * sg);
             }
           }
-        } else {
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            float ov[16];
-            tmem_ld16(tl + tOU(t % 3) + 16 * hh, ov);
-            tmem_ld_wait(ov);
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-              *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(16 * hh + r, e & 63)) = __float2bfloat16_rn(p.scale * ov[r]);
-          }
         }
         fence_proxy_async_smem();
         named_sync(kBarChain, 128);
@@ -793,7 +790,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       if (!go) break;
     }
-    if (warp == 0 && lane == 0) bulk_wait_all();
+    if (kOut && warp == 0 && lane == 0) bulk_wait_all();
     if (kOut && warp == 0 && lane == 0 && *x.abort && gate_issued >= 0)  // let the last gate copy land
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_GATE], (uint32_t)gate_issued & 1u); ++i) {
       }
@@ -907,6 +904,36 @@ __global__ void __launch_bounds__(NT, 1)
       for (int i = tt; i < 32 * 33; i += 128) N[i] = 0.f;
       named_sync(kBarTokB, 128);
     }
+    // Output tile of chunk t (plain instantiations): TMEM -> bf16 staging tile ->
+    // one TMA store, rows past the end of the sequence clipped by the tensor map.
+    // Token B takes it off the chain, two chunks behind its own work: by then the
+    // chain's dS / O MMAs of chunk t are long complete, and the TMEM slot of chunk
+    // t is next written by token B's own U product of chunk t + 3.
+    auto out_plain = [&](int t) {
+      // slot t & 1 completes once per two chunks, and chunk t + 2 cannot complete before
+      // token B has handed chunk t + 2 to the chain, so the parity below is unambiguous
+      wait_tok(x, B_OUT0 + (t & 1), (uint32_t)(t >> 1) & 1u);
+      tc_fence_after();
+      unsigned char *ot = sm + kOst + (tt >> 6) * 4096;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        float ov[16];
+        tmem_ld16(tl + tOU(t % 3) + 16 * hh, ov);
+        tmem_ld_wait(ov);
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+          *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_off(16 * hh + r, tt & 63)) = __float2bfloat16_rn(p.scale * ov[r]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_sync(kBarTokB, 128);
+      if (warp == 8) {
+        tma_store_3d_warp(&mo, sm + kOst, 0, tb + t * C, bh);
+        tma_store_3d_warp(&mo, sm + kOst + 4096, 64, tb + t * C, bh);
+        bulk_commit_warp();
+        if (lane == 0) bulk_wait_read_all();  // the tile is rewritten only after token B's next named barrier
+      }
+    };
     int v_issued = -1;  // last chunk whose v copy was issued (abort path)
     if (warp == 8 && nchunks > 0) {
       if (lane == 0) prefetch_tmap(&mv);
@@ -916,6 +943,7 @@ __global__ void __launch_bounds__(NT, 1)
     for (int t = 0; t < nchunks; ++t) {
       const int pb = t & 1;
       const float *bet = reinterpret_cast<const float *>(sm + kBeta + pb * 128);
+      if (out_b && t >= 2) out_plain(t - 2);
       wait_tok(x, B_DEC0 + pb, (uint32_t)(t >> 1) & 1u);
       wait_tok(x, B_GRAM0 + pb, (uint32_t)(t >> 1) & 1u);
       tc_fence_after();
@@ -1013,6 +1041,16 @@ __global__ void __launch_bounds__(NT, 1)
       if (tt == 0) mbar_arrive(&x.bar[B_WT0 + pb]);
       if (!go) break;
     }
+    if (out_b && nchunks > 0 && named_sync_and(kBarTokB, 128, *x.abort == 0)) {  // the last two output tiles
+      if (nchunks >= 2) {
+        out_plain(nchunks - 2);
+        // in the loop a named barrier of the chunk's own work always separates warp 8's
+        // wait for the staged tile to be read from the next tile's writes; here one is needed
+        named_sync(kBarTokB, 128);
+      }
+      out_plain(nchunks - 1);
+    }
+    if (out_b && warp == 8 && lane == 0) bulk_wait_all();
     if (tt == 0 && *x.abort && v_issued >= 0)  // let the last v copy land before the CTA exits
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&x.bar[B_V], (uint32_t)v_issued & 1u); ++i) {
       }

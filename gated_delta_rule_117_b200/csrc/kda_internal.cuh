@@ -66,6 +66,13 @@ struct SpecArgs {
   int B, H, W, dk, dv;
   int bf16;
   float scale;
+  // fused gate edges (kda_spec_replay_verify_fused; gate == null: plain loop):
+  // g holds the Eq. 5 logits z, o receives the Eq. 6 edge y
+  const float *A_log;
+  float g_min;
+  const void *gate;
+  const float *rms_w;
+  float eps;
 };
 
 cudaError_t launch_spec_replay_verify(const SpecArgs &a, cudaStream_t s);

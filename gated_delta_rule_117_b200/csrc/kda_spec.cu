@@ -156,18 +156,35 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
 // needs no barrier: the warps of a CTA run through the window independently.
 constexpr int kD = 128, kWarps = 8, kRowsPT = 16, kWB = 8;
 
-template <typename TIn>
+// kFused: the same loop with the KDA layer's gate edges folded in, as the
+// report's replay kernel does (section 5.4.2): g arrives as the Eq. 5 logits z
+// (g = g_min Sigmoid(e^A z), formed while the window is staged) and the
+// verified outputs leave as the Eq. 6 edge y = Sigmoid(gate) w o / rms(o).  The
+// RMS spans the 128 columns, i.e. all eight warps: the outputs of a staged
+// block go to shared memory and are normalised and gated after the block,
+// one barrier per block instead of one per token.
+struct SpecEdges {
+  const float *A_log;  // [H][128] Eq. 5 log-scales
+  float g_min;
+  const void *gate;    // [B][H][W][128] Eq. 6 output gate (dtype of the inputs)
+  const float *rms_w;  // [H][128] RMSNorm weights
+  float eps;
+};
+
+template <typename TIn, bool kFused>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     spec_replay_verify_d128_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                                    const TIn *__restrict__ v, const TIn *__restrict__ g,
                                    const TIn *__restrict__ beta, float *S, TIn *__restrict__ o,
-                                   const int *__restrict__ n_replay, int H, int W, float scale) {
+                                   const int *__restrict__ n_replay, int H, int W, float scale,
+                                   const SpecEdges ed) {
   const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = lane >> 2, cg = lane & 3;
   const int col4 = 4 * warp + cg;  // float4 column index of this thread (columns 4*col4 .. +3)
   // staged window block: per token and row {alpha, k} and q; v; beta; q.k
   __shared__ float2 sak[kWB][kD];
   __shared__ float sq[kWB][kD], sv[kWB][kD], sb[kWB], sqk[kWB];
+  __shared__ float so[kFused ? kWB : 1][kD];  // fused: the block's verified outputs (scaled o)
 
   const int nr = min(max(n_replay[bh / H], 0), W);
   float4 *S4 = reinterpret_cast<float4 *>(S + (size_t)bh * kD * kD);
@@ -181,7 +198,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     for (int e = tid; e < nb * kD; e += kWarps * 32) {
       const int u = e / kD, i = e % kD;
       const size_t in = ((size_t)bh * W + t0 + u) * kD + i;
-      sak[u][i] = make_float2(expf(to_f(g[in])), to_f(k[in]));
+      float gi = to_f(g[in]);
+      if (kFused) gi = __fdividef(ed.g_min, 1.f + __expf(-__expf(ed.A_log[(size_t)(bh % H) * kD + i]) * gi));
+      sak[u][i] = make_float2(expf(gi), to_f(k[in]));
       sq[u][i] = to_f(q[in]);
       sv[u][i] = to_f(v[in]);
     }
@@ -249,11 +268,37 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
         for (int r = 0; r < kRowsPT; ++r) S4[(rg + 8 * r) * (kD / 4) + col4] = s[r];
       if (out && rg == 0) {
         const float qk = sqk[u];
-        TIn *ob = o + ((size_t)bh * W + t) * kD + 4 * col4;
-        put(ob + 0, scale * (r0.x + qk * u0.x));
-        put(ob + 1, scale * (r0.y + qk * u0.y));
-        put(ob + 2, scale * (r1.x + qk * u1.x));
-        put(ob + 3, scale * (r1.y + qk * u1.y));
+        const float4 ov = make_float4(scale * (r0.x + qk * u0.x), scale * (r0.y + qk * u0.y),
+                                      scale * (r1.x + qk * u1.x), scale * (r1.y + qk * u1.y));
+        if (kFused) {
+          *reinterpret_cast<float4 *>(&so[kFused ? u : 0][4 * col4]) = ov;
+        } else {
+          TIn *ob = o + ((size_t)bh * W + t) * kD + 4 * col4;
+          put(ob + 0, ov.x);
+          put(ob + 1, ov.y);
+          put(ob + 2, ov.z);
+          put(ob + 3, ov.w);
+        }
+      }
+    }
+    if (kFused) {
+      // Eq. 6 edge of the block's verified outputs: one warp per token, four columns per lane
+      __syncthreads();
+      for (int u = warp; u < nb; u += kWarps) {
+        const int t = t0 + u;
+        if (t < nr) continue;
+        const float4 ov = *reinterpret_cast<const float4 *>(&so[kFused ? u : 0][4 * lane]);
+        float ss = (ov.x * ov.x + ov.y * ov.y) + (ov.z * ov.z + ov.w * ov.w);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rinv = rsqrtf(ss * (1.f / kD) + ed.eps);
+        const size_t at = ((size_t)bh * W + t) * kD + 4 * lane;
+        const TIn *gt = reinterpret_cast<const TIn *>(ed.gate) + at;
+        const float *wv = ed.rms_w + (size_t)(bh % H) * kD + 4 * lane;
+        const float y[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          put(o + at + j, y[j] * rinv * wv[j] * __fdividef(1.f, 1.f + __expf(-to_f(gt[j]))));
       }
     }
   }
@@ -270,11 +315,18 @@ cudaError_t launch_t(const SpecArgs &a, cudaStream_t st) {
 template <typename TIn>
 cudaError_t launch_dt(const SpecArgs &a, cudaStream_t st) {
   if (a.dk == kD && a.dv == kD) {
-    spec_replay_verify_d128_kernel<TIn><<<a.B * a.H, kWarps * 32, 0, st>>>(
-        (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
-        (TIn *)a.o, a.n_replay, a.H, a.W, a.scale);
+    const SpecEdges ed{a.A_log, a.g_min, a.gate, a.rms_w, a.eps};
+    if (a.gate)
+      spec_replay_verify_d128_kernel<TIn, true><<<a.B * a.H, kWarps * 32, 0, st>>>(
+          (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
+          (TIn *)a.o, a.n_replay, a.H, a.W, a.scale, ed);
+    else
+      spec_replay_verify_d128_kernel<TIn, false><<<a.B * a.H, kWarps * 32, 0, st>>>(
+          (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
+          (TIn *)a.o, a.n_replay, a.H, a.W, a.scale, ed);
     return cudaGetLastError();
   }
+  if (a.gate) return cudaErrorInvalidValue;  // the fused edges exist for dk = dv = 128 only
 #define KDA_SP_CASE(DKv, DVv) \
   if (a.dk == DKv && a.dv == DVv) return launch_t<DKv, DVv, TIn>(a, st);
 #define KDA_SP_ROW(DKv) KDA_SP_CASE(DKv, 16) KDA_SP_CASE(DKv, 32) KDA_SP_CASE(DKv, 64) KDA_SP_CASE(DKv, 128)

@@ -26,7 +26,7 @@ EXPORTED = ["kda_chunk_fwd_plan", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd
             "kda_status_string", "kda_get_device_status", "kda_version", "kda_chunk_fwd_noalloc",
             "kda_noalloc_scratch_bytes", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_gated", "kda_output_gate",
             "kda_kcp_compose", "kda_spec_replay_verify", "kda_debug_set_wait_limit", "kda_debug_inject_stall",
-            "kda_chunk_fwd_outgate", "kda_chunk_transition"]
+            "kda_chunk_fwd_outgate", "kda_chunk_transition", "kda_spec_replay_verify_fused"]
 
 
 class KdaError(RuntimeError):
@@ -73,6 +73,8 @@ def load_library():
             lib.kda_output_gate.restype = i
             lib.kda_kcp_compose.argtypes = [vp] * 4 + [i] * 5 + [vp]
             lib.kda_kcp_compose.restype = i
+            lib.kda_spec_replay_verify_fused.argtypes = [vp] * 5 + [f] + [vp] * 4 + [f] + [vp] * 2 + [i] * 6 + [f, vp]
+            lib.kda_spec_replay_verify_fused.restype = i
             lib.kda_spec_replay_verify.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
             lib.kda_spec_replay_verify.restype = i
             lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
@@ -168,6 +170,14 @@ def kda_spec_replay_verify(q, k, v, g, beta, S, o, n_replay, B, H, W, dk, dv, dt
     """Speculative-decode replay and verify over a W-token window.  Returns the raw kda_status_t."""
     return load_library().kda_spec_replay_verify(q, k, v, g, beta, S, o, n_replay, B, H, W, dk, dv, dtype, scale,
                                                  stream)
+
+
+def kda_spec_replay_verify_fused(q, k, v, z, A_log, g_min, beta, S, gate, rms_weight, eps, y, n_replay, B, H, W, dk,
+                                 dv, dtype, scale, stream) -> int:
+    """The replay loop with the Eq. 5 gate (z, A_log) and the Eq. 6 edge (gate,
+    rms_weight -> y) folded in.  Returns the raw kda_status_t."""
+    return load_library().kda_spec_replay_verify_fused(q, k, v, z, A_log, g_min, beta, S, gate, rms_weight, eps, y,
+                                                       n_replay, B, H, W, dk, dv, dtype, scale, stream)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, h0, o, h_T, B, H, T, dk, dv, dtype, chunk_size, scale, stream) -> int:
@@ -378,3 +388,21 @@ def recurrent_step(q, k, v, g, beta, S, *, o=None, scale=0.0, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_recurrent_step")
     return o
+
+
+def spec_replay_verify_fused(q, k, v, z, A_log, beta, S, gate, rms_weight, n_replay, *, g_min=-5.0, eps=1e-6, y=None,
+                             scale=0.0, stream=None):
+    """spec_replay_verify with the Eq. 5 gate on the inputs (z [B, H, W, dk],
+    A_log [H, dk] fp32) and the Eq. 6 edge on the verified outputs (gate
+    [B, H, W, dv], rms_weight [H, dv] fp32).  Returns y (zeros for replayed tokens)."""
+    import torch
+    B, H, W, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.zeros(B, H, W, dv, dtype=q.dtype, device=q.device)
+    st = kda_spec_replay_verify_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta),
+                                      _ptr(S), _ptr(gate), _ptr(rms_weight), float(eps), _ptr(y), _ptr(n_replay), B, H,
+                                      W, dk, dv, _dtype_code(q), float(scale), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_spec_replay_verify_fused")
+    return y

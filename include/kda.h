@@ -292,6 +292,28 @@ kda_status_t kda_spec_replay_verify(const void *q, const void *k, const void *v,
                                     kda_stream_t stream);
 
 /*
+ * The replay loop with the KDA layer's gate edges folded in (Kimi K3 report,
+ * section 5.4.2: one fused loop over replayed, bonus and draft tokens; the
+ * gates of section 2.1.1, Eq. 5 and Eq. 6).  Same window, state and replay
+ * semantics as kda_spec_replay_verify, except that
+ *   z     : [B, H, W, dk] the Eq. 5 decay logits in place of g;
+ *           g = g_min * Sigmoid(exp(A_log) * z) is formed on chip
+ *   A_log : [H, dk] fp32;   g_min in [-5, 0)
+ *   gate  : [B, H, W, dv] (dtype) the Eq. 6 output gate;  rms_weight : [H, dv] fp32;  eps >= 0
+ *   y     : [B, H, W, dv] (dtype), written for the verified tokens (t >= n_replay[b]) only:
+ *           y_t = Sigmoid(gate_t) * rms_weight * o_t / sqrt(mean(o_t^2) + eps)
+ * dk = dv = 128 only (KDA_ERR_SHAPE otherwise).  The short convolution and
+ * input normalisation of the report's loop need the layer's projection and
+ * convolution weights and are not part of this call.  y, S must not overlap
+ * any input (gate, A_log, rms_weight included).
+ */
+kda_status_t kda_spec_replay_verify_fused(const void *q, const void *k, const void *v, const void *z,
+                                          const float *A_log, float g_min, const void *beta, float *S,
+                                          const void *gate, const float *rms_weight, float eps, void *y,
+                                          const int *n_replay, int B, int H, int W, int dk, int dv,
+                                          kda_dtype_t dtype, float scale, kda_stream_t stream);
+
+/*
  * Prefill without a caller-provided workspace, for callers that cannot
  * allocate device memory (e.g. a plugin inside a host framework that owns the
  * GPU memory pool and exposes no allocator, or a latency-critical path where

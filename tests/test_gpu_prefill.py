@@ -260,3 +260,23 @@ def test_misaligned_pointer_is_rejected():
         kda.chunk_fwd(qm, d["k"], d["v"], d["g"], d["beta"], None)
     assert e.value.status == 4
     assert kda.kda_get_device_status() == 0
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 16, 4096), (4, 37, 700)])
+def test_back_to_back_calls_record_no_timeout(B, H, T):
+    # the roles of the tensor-core kernel hand chunks over through mbarrier phases;
+    # a wait on a phase that can alias (complete twice before it is observed) stalls
+    # until its bounded wait gives up.  Such a race is timing-dependent, so run many
+    # calls back to back and require that none recorded a timeout, and that the
+    # calls take normal time (a stall costs the 2 s wait limit)
+    import time
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=B, H=H, T=T, seed=131)
+    d = to_dev(synth.prefill_inputs(w))
+    o, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"])
+    assert kda.kda_get_device_status() == 0
+    t0 = time.perf_counter()
+    for _ in range(40):
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], o=o, h_T=hT)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    assert time.perf_counter() - t0 < 1.0

@@ -60,3 +60,36 @@ def test_replay_then_verify_equals_stepwise_decode():
         kda.recurrent_step(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], S_b)
     torch.cuda.synchronize()
     assert rel_l2(S_a, S_b) <= 1e-6
+
+
+@pytest.mark.parametrize("dtype,key", [("bf16", "bf16"), ("f32", "f32")])
+def test_fused_gate_edges_in_the_replay_loop(dtype, key):
+    # the replay loop with the Eq. 5 gate on the inputs and the Eq. 6 edge on the
+    # verified outputs: against oracle.gate -> oracle.recurrent -> oracle.output_gate
+    W = 6
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=3, H=2, T=W, dtype=dtype, seed=84)
+    x = synth.prefill_inputs(w)
+    gi = synth.gate_inputs(w)
+    g = torch.Generator().manual_seed(85)
+    gate = (2 * torch.randn(w.B, w.H, W, 128, generator=g)).to(w.torch_dtype)
+    rw = (1 + 0.3 * torch.randn(w.H, 128, generator=g)).float()
+    n_replay = [0, 2, 6]
+    d = {n: t.cuda() for n, t in x.items()}
+    S = d["h0"].clone()
+    nr = torch.tensor(n_replay, dtype=torch.int32, device="cuda")
+    y = kda.spec_replay_verify_fused(d["q"], d["k"], d["v"], gi["z"].cuda(), gi["A_log"].cuda(), d["beta"], S,
+                                     gate.cuda(), rw.cuda(), nr, eps=1e-6)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    g_ref = oracle.gate(f64(gi["z"]), gi["A_log"].double().numpy())
+    a = [f64(x["q"]), f64(x["k"]), f64(x["v"]), g_ref, f64(x["beta"])]
+    o_ref, _ = oracle.recurrent(*a, f64(x["h0"]))
+    y_ref = oracle.output_gate(o_ref, f64(gate), rw.double().numpy(), 1e-6)
+    for b, n in enumerate(n_replay):
+        if n > 0:
+            _, s_ref = oracle.recurrent(*[t[b:b + 1, :, :n] for t in a], f64(x["h0"])[b:b + 1])
+        else:
+            s_ref = f64(x["h0"])[b:b + 1]
+        assert rel_l2(S[b:b + 1], s_ref) <= 1e-5, (b, n)
+        if n < W:
+            assert rel_l2(y[b:b + 1, :, n:], y_ref[b:b + 1, :, n:]) <= TOL[key], (b, n)
