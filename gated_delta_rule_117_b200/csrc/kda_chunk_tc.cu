@@ -187,6 +187,8 @@ struct TcParams {
   const float *rms_w;  // [H][128] RMSNorm weights of the fused Eq. 6 edge (the gate map holds its gate)
   float eps;
   int m_rowmajor;  // transition runs: M stored row-major (1) or transposed for the segment scan (0)
+  unsigned *m_vanished;  // [BH][nseg-1] (in-device CP): 1 where the M run ended on an all-zero state
+                         // (its stored M is exactly zero), else 0; null outside the segmented plan
 };
 
 struct Ctx {
@@ -1065,6 +1067,10 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // in-device CP: tell the scan whether this M run ended on an all-zero state (its
+  // stored M is then exactly zero and the scan need not load or apply it)
+  if (kTrans && kind == 2 && p.m_vanished && tid == 0)
+    p.m_vanished[(size_t)bh * (p.nseg - 1) + seg] = (*x.abort == kFinishedEarly) ? 1u : 0u;
   if (warp == 4) {
     bool drained = false;
     for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(&x.bar[B_DRAIN], 0u);
@@ -1080,8 +1086,11 @@ __global__ void __launch_bounds__(NT, 1)
 // The transitions arrive transposed (MT[k][i] = M[i][k]), so a warp reading
 // M[i][k] for 16 consecutive rows i touches 16 consecutive words; the next
 // transition is loaded into registers while the current one is applied.
+// A transition that vanished (the M run ended on an all-zero state, so M = 0
+// exactly) is neither loaded nor applied: S_in(s+1) = S~_s, bit for bit what
+// the product with a zero M gives.
 __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const float *MT, const float *St, float *Sin,
-                                                      int nseg) {
+                                                      const unsigned *vanished, int nseg) {
   extern __shared__ float cps[];
   float *Ms = cps;               // [128 k][128 i]
   float *X = cps + D * D;        // [128][16]
@@ -1090,10 +1099,14 @@ __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const flo
   const int i = 2 * (tid >> 2), j0 = 4 * (tid & 3);
   const size_t mat = (size_t)D * D;
   float4 pre[16], spre[2];
+  bool vnext = false;  // the prefetched segment's transition vanished
   auto fetch = [&](int s) {
+    vnext = __ldg(vanished + (size_t)bh * (nseg - 1) + s) != 0u;
     const float4 *Mg = reinterpret_cast<const float4 *>(MT + ((size_t)bh * (nseg - 1) + s) * mat);
+    if (!vnext) {
 #pragma unroll
-    for (int u = 0; u < 16; ++u) pre[u] = __ldg(Mg + tid + 256 * u);
+      for (int u = 0; u < 16; ++u) pre[u] = __ldg(Mg + tid + 256 * u);
+    }
     const float *Sg = St + ((size_t)bh * (nseg - 1) + s) * mat + (size_t)i * D + c0 + j0;
     spre[0] = __ldg(reinterpret_cast<const float4 *>(Sg));
     spre[1] = __ldg(reinterpret_cast<const float4 *>(Sg + D));
@@ -1112,15 +1125,18 @@ __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const flo
       *reinterpret_cast<float4 *>(X + (i + r) * 16 + j0) = acc[r];
     }
     if (s + 1 >= nseg) break;
+    const bool vz = vnext;  // segment s's transition vanished (uniform over the CTA)
+    if (!vz) {
 #pragma unroll
-    for (int u = 0; u < 16; ++u) reinterpret_cast<float4 *>(Ms)[tid + 256 * u] = pre[u];
+      for (int u = 0; u < 16; ++u) reinterpret_cast<float4 *>(Ms)[tid + 256 * u] = pre[u];
+    }
     // packed accumulators: (row, columns 0-1) and (row, columns 2-3)
     float2 a00 = make_float2(spre[0].x, spre[0].y), a01 = make_float2(spre[0].z, spre[0].w);
     float2 a10 = make_float2(spre[1].x, spre[1].y), a11 = make_float2(spre[1].z, spre[1].w);
     __syncthreads();
     if (s + 2 < nseg) fetch(s + 1);
 #pragma unroll 8
-    for (int k = 0; k < D; ++k) {
+    for (int k = 0; k < (vz ? 0 : D); ++k) {
       const float2 m = *reinterpret_cast<const float2 *>(Ms + k * D + i);  // M[i][k], M[i+1][k]
       const float4 xv = *reinterpret_cast<const float4 *>(X + k * 16 + j0);
       const float2 xlo = make_float2(xv.x, xv.y), xhi = make_float2(xv.z, xv.w);
@@ -1162,7 +1178,8 @@ size_t tc32_workspace(int BH, int T) {
   const int P = tc32_segments(BH, T);
   if (P <= 1) return 0;
   const size_t mat = (size_t)D * D * sizeof(float);
-  return (size_t)BH * (2 * (P - 1) + P) * mat;
+  const size_t flags = ((size_t)BH * (P - 1) * sizeof(unsigned) + 15) / 16 * 16;
+  return (size_t)BH * (2 * (P - 1) + P) * mat + flags;
 }
 
 cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
@@ -1201,6 +1218,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.rms_w = a.rms_w;
   p.eps = a.eps;
   p.m_rowmajor = 0;
+  p.m_vanished = nullptr;
   const bool gated = a.A_log != nullptr;
   // one variant per call: checkpoints, the fused gate and the fused output edge do not combine
   if ((p.ckpt != nullptr) + (int)gated + (int)out_edge > 1) return cudaErrorInvalidValue;
@@ -1246,9 +1264,11 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   if (P2 != P) return cudaErrorInvalidValue;
   p.seg_len = L;
   p.nseg = P;
+  unsigned *vanished = reinterpret_cast<unsigned *>(Sin + (size_t)BH * P * mat);
   p.m_out = Mw;
   p.st_out = Sw;
   p.sin = Sin;
+  p.m_vanished = vanished;
   p.mode = kModeSegTransition;
   float *const ckpt = p.ckpt;
   p.ckpt = nullptr;  // transition runs start from 0 or I: no checkpoints there
@@ -1260,7 +1280,8 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
     return e;
-  cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, P);
+  cp_scan_kernel<<<dim3(BH, 8), 256, scan_smem, st>>>(a.h0, Mw, Sw, Sin, vanished, P);
+  p.m_vanished = nullptr;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.mode = kModeSegFinal;
   p.ckpt = ckpt;

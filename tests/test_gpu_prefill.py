@@ -94,6 +94,21 @@ def test_in_device_context_parallel(B, H, T):
     assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("g_scale", [1.0, 0.05])
+def test_in_device_context_parallel_vanishing_and_persistent_transitions(g_scale):
+    # at the workloads' decay every segment's transition M underflows to exactly zero
+    # (the M runs stop early and the scan skips them); with decays 20x slower M stays
+    # nonzero over a 256-token segment (~e^-32) and the scan multiplies by it
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=8, T=2304, seed=141)
+    x = synth.prefill_inputs(w)
+    x["g"] = (x["g"].float() * g_scale).to(x["g"].dtype)
+    plan = kda.kda_chunk_fwd_plan(1, 8, 2304, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    assert plan["segments"] > 1
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
 def test_context_parallel_inplace_state_and_missing_workspace():
     w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=8, T=1024, seed=5)
     x = synth.prefill_inputs(w)
