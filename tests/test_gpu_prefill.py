@@ -258,12 +258,16 @@ def test_state_split_resume_on_gpu():
     assert rel_l2(h2, h_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
 
 
-def test_deterministic():
-    w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=300, H=4)
+@pytest.mark.parametrize("T", [300, 1100])  # one CTA per chain; segmented plan
+def test_deterministic(T):
+    # the roles hand data over through shared and tensor memory; a missing wait or
+    # barrier usually shows up as run-to-run differences, so results must be bitwise stable
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(T=T, H=4)
     x = synth.prefill_inputs(w)
     o1, h1 = _run(x)
-    o2, h2 = _run(x)
-    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    for _ in range(3):
+        o2, h2 = _run(x)
+        assert torch.equal(o1, o2) and torch.equal(h1, h2)
 
 
 def test_misaligned_pointer_is_rejected():
