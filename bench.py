@@ -348,9 +348,9 @@ def prefill_figures(w, plan, ms, pk, pk_kind, synth):
     flop_tok = synth.flops_per_token_head(dk, dv, 64)
     tflops = flop_tok * B * H * T / (ms / 1e3) / 1e12
     kernel = "chunk16_kernel" if plan["path"] == 1 else "chunk_tc_kernel"
-    # With in-device context parallelism one step is three launches (segment
-    # transitions, the prefix scan, the final pass); the roofline then uses the
-    # whole step's time, which is the conservative reading.
+    # With in-device context parallelism one step is four launches (the two
+    # segment-transition passes, the prefix scan, the final pass); the roofline
+    # then uses the whole step's time, which is the conservative reading.
     scope = "kernel" if plan["launches"] == 1 else "step (%d launches)" % plan["launches"]
     src = (["gated_delta_rule_117_b200/csrc/kda_chunk_simt.cu"] if plan["path"] == 1
            else ["gated_delta_rule_117_b200/csrc/kda_chunk_tc.cu"])

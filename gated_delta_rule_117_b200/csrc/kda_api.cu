@@ -108,7 +108,7 @@ kda_status_t plan_prefill(int B, int H, int T, int dk, int dv, kda_dtype_t dtype
   p.segments = 1;
   if (tc) kda::tc32_plan(B * H, T, &p.segments, &seg_len);
   p.segment_tokens = p.segments > 1 ? seg_len : T;
-  p.launches = (B * H == 0) ? 0 : (p.segments > 1 ? 3 : 1);
+  p.launches = (B * H == 0) ? 0 : (p.segments > 1 ? 4 : 1);
   p.workspace = tc ? kda::tc32_workspace(B * H, T) : 0;
   *plan = p;
   return KDA_OK;

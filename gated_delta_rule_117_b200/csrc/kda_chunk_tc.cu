@@ -189,6 +189,9 @@ struct TcParams {
   int m_rowmajor;  // transition runs: M stored row-major (1) or transposed for the segment scan (0)
   unsigned *m_vanished;  // [BH][nseg-1] (in-device CP): 1 where the M run ended on an all-zero state
                          // (its stored M is exactly zero), else 0; null outside the segmented plan
+  int win;               // transition runs: tokens before the segment's end that they cover (0: all)
+  unsigned *win_final;   // [BH][nseg-1] window pass: 1 where the window's result is the segment's own
+  const unsigned *skip;  // [BH][nseg-1] second transition pass: segments that need no full run
 };
 
 struct Ctx {
@@ -488,8 +491,10 @@ __global__ void __launch_bounds__(NT, 1)
     bh = blockIdx.x / p.nseg;
     seg = blockIdx.x % p.nseg;
   }
-  const int tb = seg * p.seg_len;
-  const int te = min(T, tb + p.seg_len);
+  const int te = min(T, seg * p.seg_len + p.seg_len);
+  // a transition run covers its whole segment, or the window of p.win tokens before its end
+  const int tb = kTrans && p.win > 0 ? max(seg * p.seg_len, te - p.win) : seg * p.seg_len;
+  if (kTrans && p.skip && p.skip[(size_t)bh * (p.nseg - 1) + seg]) return;  // the window's result stands
   const int nchunks = (te - tb + C - 1) / C;
   const bool v_zero = kTrans && kind == 2;
   const bool store_o = !kTrans;
@@ -701,8 +706,10 @@ __global__ void __launch_bounds__(NT, 1)
       // the run stops, like an abort but without an error, and stores those
       // zeros -- the result this kernel would have computed over the rest of
       // the segment, bit for bit.  Under decaying gates the state vanishes
-      // within a few chunks; a state that does not vanish runs to the end.
-      if (kTrans && v_zero && has_next) {
+      // within a few chunks; a state that does not vanish runs to the end.  (The
+      // window pass checks after its last chunk too: the flag it leaves decides
+      // whether the segment runs again in full.)
+      if (kTrans && v_zero && (has_next || p.win > 0)) {
         uint32_t bits = 0;
 #pragma unroll
         for (int i = 0; i < D / 2; ++i) bits |= (__float_as_uint(S[i].x) | __float_as_uint(S[i].y)) & 0x7fffffffu;
@@ -1069,8 +1076,14 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   // in-device CP: tell the scan whether this M run ended on an all-zero state (its
   // stored M is then exactly zero and the scan need not load or apply it)
-  if (kTrans && kind == 2 && p.m_vanished && tid == 0)
-    p.m_vanished[(size_t)bh * (p.nseg - 1) + seg] = (*x.abort == kFinishedEarly) ? 1u : 0u;
+  if (kTrans && kind == 2 && tid == 0) {
+    const size_t slot = (size_t)bh * (p.nseg - 1) + seg;
+    const bool vanished = *x.abort == kFinishedEarly;
+    if (p.m_vanished) p.m_vanished[slot] = vanished ? 1u : 0u;
+    // the window's (S~, M) are the segment's own when the window is the whole segment,
+    // or when M vanished over it (see the window pass in launch_chunk_tc32)
+    if (p.win_final) p.win_final[slot] = (vanished || tb == seg * p.seg_len) ? 1u : 0u;
+  }
   if (warp == 4) {
     bool drained = false;
     for (uint32_t i = 0; i < kWaitLimit && !drained; ++i) drained = mbar_try_wait(&x.bar[B_DRAIN], 0u);
@@ -1153,6 +1166,9 @@ __global__ void __launch_bounds__(256) cp_scan_kernel(const float *h0, const flo
 
 }  // namespace
 
+// tokens before a segment's end covered by the first transition pass (see launch_chunk_tc32)
+constexpr int kTransWindow = 4 * C;
+
 void tc32_plan(int BH, int T, int *segments, int *seg_len) {
   // Fill the 148 SMs (one CTA each) when there are few chains; segments of at
   // least 256 tokens keep the extra passes worthwhile.  Segment lengths are
@@ -1178,7 +1194,7 @@ size_t tc32_workspace(int BH, int T) {
   const int P = tc32_segments(BH, T);
   if (P <= 1) return 0;
   const size_t mat = (size_t)D * D * sizeof(float);
-  const size_t flags = ((size_t)BH * (P - 1) * sizeof(unsigned) + 15) / 16 * 16;
+  const size_t flags = (2 * (size_t)BH * (P - 1) * sizeof(unsigned) + 15) / 16 * 16;
   return (size_t)BH * (2 * (P - 1) + P) * mat + flags;
 }
 
@@ -1219,6 +1235,9 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.eps = a.eps;
   p.m_rowmajor = 0;
   p.m_vanished = nullptr;
+  p.win = 0;
+  p.win_final = nullptr;
+  p.skip = nullptr;
   const bool gated = a.A_log != nullptr;
   // one variant per call: checkpoints, the fused gate and the fused output edge do not combine
   if ((p.ckpt != nullptr) + (int)gated + (int)out_edge > 1) return cudaErrorInvalidValue;
@@ -1265,6 +1284,7 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.seg_len = L;
   p.nseg = P;
   unsigned *vanished = reinterpret_cast<unsigned *>(Sin + (size_t)BH * P * mat);
+  unsigned *win_final = vanished + (size_t)BH * (P - 1);
   p.m_out = Mw;
   p.st_out = Sw;
   p.sin = Sin;
@@ -1272,11 +1292,30 @@ cudaError_t launch_chunk_tc32(const ChunkArgs &a, cudaStream_t st) {
   p.mode = kModeSegTransition;
   float *const ckpt = p.ckpt;
   p.ckpt = nullptr;  // transition runs start from 0 or I: no checkpoints there
-  if (gated)
-    chunk_tc_kernel<false, true, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
-  else
-    chunk_tc_kernel<false, false, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  auto launch_transition = [&]() {
+    if (gated)
+      chunk_tc_kernel<false, true, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    else
+      chunk_tc_kernel<false, false, true, false><<<BH * 2 * (P - 1), NT, kSmemBytes, st>>>(mq, mk, mv, mg, mo, mgate, p);
+    return cudaGetLastError();
+  };
+  // Window pass: every segment's (S~, M) over its last kTransWindow tokens only.
+  // Split a segment at the window's start: Eq. 17 gives M = M_tail M_head and
+  // S~ = M_tail S~_head + S~_tail.  Where the window's M run ends on an exactly
+  // zero state (an fp32 underflow; at the workloads' decay, g ~ -2.5 per token,
+  // within two chunks), M_tail is zero to fp32's range, so the segment's M is
+  // zero and its S~ is the window's S~_tail: the terms dropped lie below fp32's
+  // underflow threshold.  The scan then never reads M (the vanished flag).
+  p.win = kTransWindow;
+  p.win_final = win_final;
+  if ((e = launch_transition()) != cudaSuccess) return e;
+  // Second pass: the whole segment, only where the window's M did not vanish (slow
+  // decay); every other CTA returns at once.
+  p.win = 0;
+  p.win_final = nullptr;
+  p.skip = win_final;
+  if ((e = launch_transition()) != cudaSuccess) return e;
+  p.skip = nullptr;
   const int scan_smem = (128 * 128 + 128 * 16) * (int)sizeof(float);
   if ((e = cudaFuncSetAttribute(cp_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem)) != cudaSuccess)
     return e;

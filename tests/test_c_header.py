@@ -44,7 +44,7 @@ def test_c_program_against_the_library(tmp_path):
                            "-L", PKG, "-lkda", "-Wl,-rpath," + PKG, "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
     status, path, chunk, segments, launches, workspace = map(int, out[0].split())
-    assert status == 0 and path == 2 and chunk == 32 and segments == 9 and launches == 3 and workspace > 0
+    assert status == 0 and path == 2 and chunk == 32 and segments == 9 and launches == 4 and workspace > 0
     assert int(out[1]) == 2                              # KDA_ERR_SHAPE for dk = 24
     assert out[2].startswith("KDA_ERR_ALIAS")
     assert int(out[3]) >= 100

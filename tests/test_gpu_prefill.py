@@ -87,7 +87,7 @@ def test_in_device_context_parallel(B, H, T):
     # (transition pass, scan, final pass); results must match the recurrence
     w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=B, H=H, T=T, seed=123)
     plan = kda.kda_chunk_fwd_plan(B, H, T, 128, 128, kda.KDA_DTYPE_BF16, 0)
-    assert plan["segments"] > 1 and plan["launches"] == 3 and plan["workspace"] > 0
+    assert plan["segments"] > 1 and plan["launches"] == 4 and plan["workspace"] > 0
     x = synth.prefill_inputs(w)
     o, hT = _run(x)
     o_ref, h_ref = oracle_prefill(x)
@@ -107,6 +107,30 @@ def test_in_device_context_parallel_vanishing_and_persistent_transitions(g_scale
     o, hT = _run(x)
     o_ref, h_ref = oracle_prefill(x)
     assert rel_l2(o, o_ref) <= TOL["bf16"] and rel_l2(hT, h_ref) <= TOL["bf16"]
+
+
+def test_in_device_context_parallel_transition_windows():
+    # The first transition pass covers only the last 128 tokens of each 256-token
+    # segment; a segment whose window transition vanished keeps the window's (S~, M),
+    # the others run again in full.  Per head: both halves fast (window final);
+    # both slow (full run, M persists); fast head, slow window (full run, whose M
+    # vanishes); slow head, fast window (window final).  Each head must match the
+    # oracle on its own.
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=1, H=4, T=2304, seed=143)
+    plan = kda.kda_chunk_fwd_plan(1, 4, 2304, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    assert plan["segments"] == 9 and plan["segment_tokens"] == 256
+    x = synth.prefill_inputs(w)
+    in_window = (torch.arange(w.T) % 256) >= 128
+    scale = torch.ones(w.H, w.T)
+    scale[1] = 0.05
+    scale[2, in_window] = 0.05
+    scale[3, ~in_window] = 0.05
+    x["g"] = (x["g"].float() * scale[None, :, :, None]).to(x["g"].dtype)
+    o, hT = _run(x)
+    o_ref, h_ref = oracle_prefill(x)
+    for h in range(w.H):
+        assert rel_l2(o[:, h], o_ref[:, h]) <= TOL["bf16"], h
+        assert rel_l2(hT[:, h], h_ref[:, h]) <= TOL["bf16"], h
 
 
 def test_context_parallel_inplace_state_and_missing_workspace():
