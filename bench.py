@@ -426,6 +426,7 @@ def main():
     ap.add_argument("--no-subconfigs", action="store_true", help="skip the other prefill workloads")
     ap.add_argument("--no-legs", action="store_true", help="skip the secondary legs (ckpt, gates, replay)")
     ap.add_argument("--decode-only", action="store_true", help="only the decode measurement (for profiling)")
+    ap.add_argument("--spec-only", action="store_true", help="only the replay-window measurement (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -473,6 +474,9 @@ def main():
 
     if args.decode_only:
         print(json.dumps(measure_decode(args, synth, kda, torch, dev, pk, pk_kind)))
+        return
+    if args.spec_only:
+        print(json.dumps(measure_spec(args, synth, kda, torch, dev, pk)))
         return
     d = {k: v.to(dev) for k, v in x.items()}
     h0 = d["h0"] if w.h0_std > 0 else None

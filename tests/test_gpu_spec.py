@@ -93,3 +93,62 @@ def test_fused_gate_edges_in_the_replay_loop(dtype, key):
         assert rel_l2(S[b:b + 1], s_ref) <= 1e-5, (b, n)
         if n < W:
             assert rel_l2(y[b:b + 1, :, n:], y_ref[b:b + 1, :, n:]) <= TOL[key], (b, n)
+
+
+def test_many_chains_per_cta_and_two_staged_blocks():
+    # more chains than the SMs hold at once (several waves of CTAs); W = 11 spans two
+    # staged blocks of 8 tokens
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=24, H=16, T=11, seed=86)
+    assert w.B * w.H > 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    _check(w, [(5 * b) % 13 for b in range(w.B)], "bf16")  # 0 .. 12: none, some, all, clamped
+
+
+def test_fused_many_chains():
+    W = 3
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=20, H=16, T=W, seed=87)
+    x = synth.prefill_inputs(w)
+    gi = synth.gate_inputs(w)
+    g = torch.Generator().manual_seed(88)
+    gate = (2 * torch.randn(w.B, w.H, W, 128, generator=g)).to(w.torch_dtype)
+    rw = (1 + 0.3 * torch.randn(w.H, 128, generator=g)).float()
+    n_replay = [b % 4 for b in range(w.B)]
+    d = {n: t.cuda() for n, t in x.items()}
+    S = d["h0"].clone()
+    nr = torch.tensor(n_replay, dtype=torch.int32, device="cuda")
+    y = kda.spec_replay_verify_fused(d["q"], d["k"], d["v"], gi["z"].cuda(), gi["A_log"].cuda(), d["beta"], S,
+                                     gate.cuda(), rw.cuda(), nr, eps=1e-6)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    g_ref = oracle.gate(f64(gi["z"]), gi["A_log"].double().numpy())
+    a = [f64(x["q"]), f64(x["k"]), f64(x["v"]), g_ref, f64(x["beta"])]
+    o_ref, _ = oracle.recurrent(*a, f64(x["h0"]))
+    y_ref = oracle.output_gate(o_ref, f64(gate), rw.double().numpy(), 1e-6)
+    for b, n in enumerate(n_replay):
+        s_ref = (oracle.recurrent(*[t[b:b + 1, :, :n] for t in a], f64(x["h0"])[b:b + 1])[1] if n > 0
+                 else f64(x["h0"])[b:b + 1])
+        assert rel_l2(S[b:b + 1], s_ref) <= 1e-5, (b, n)
+        if n < W:
+            assert rel_l2(y[b:b + 1, :, n:], y_ref[b:b + 1, :, n:]) <= TOL["bf16"], (b, n)
+
+
+def test_inputs_off_16_byte_boundaries():
+    # window inputs that start 2 bytes past a 16-byte boundary (element-aligned only)
+    # must give bitwise the same result as aligned ones
+    w = synth.WORKLOADS["prefill_h16_t4k"].with_(B=3, H=4, T=5, seed=89)
+    x = synth.prefill_inputs(w)
+    d = {n: t.cuda() for n, t in x.items()}
+    nr = torch.tensor([0, 2, 5], dtype=torch.int32, device="cuda")
+    S_a = d["h0"].clone()
+    o_a = kda.spec_replay_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], S_a, nr)
+    shifted = {}
+    for n in ("q", "k", "v", "g"):
+        buf = torch.empty(d[n].numel() + 1, dtype=d[n].dtype, device="cuda")
+        view = buf[1:].view(d[n].shape)
+        view.copy_(d[n])
+        assert view.data_ptr() % 16 != 0
+        shifted[n] = view
+    S_b = d["h0"].clone()
+    o_b = kda.spec_replay_verify(shifted["q"], shifted["k"], shifted["v"], shifted["g"], d["beta"], S_b, nr)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    assert torch.equal(S_a, S_b) and torch.equal(o_a, o_b)
