@@ -171,16 +171,25 @@ struct SpecEdges {
   float eps;
 };
 
-template <typename TIn, bool kFused>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+// kSplit: CTAs per chain.  The recurrence is independent across value columns
+// (a column of S needs only k, g, beta and its own v), so the plain loop runs
+// each chain as two CTAs of 64 columns: four smaller CTAs per SM instead of two
+// overlap one CTA's state transfers with another's window better (each stages
+// the window's q, k, g in full).  The fused loop keeps one CTA per chain: its
+// RMS spans all 128 columns.
+template <typename TIn, bool kFused, int kSplit>
+__global__ void __launch_bounds__(kWarps * 32 / kSplit, 2 * kSplit)
     spec_replay_verify_d128_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                                    const TIn *__restrict__ v, const TIn *__restrict__ g,
                                    const TIn *__restrict__ beta, float *S, TIn *__restrict__ o,
                                    const int *__restrict__ n_replay, int H, int W, float scale,
                                    const SpecEdges ed) {
-  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  static_assert(!kFused || kSplit == 1, "the fused edge needs every column of a token in one CTA");
+  constexpr int kW = kWarps / kSplit;  // warps of this CTA
+  const int bh = blockIdx.x / kSplit, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = lane >> 2, cg = lane & 3;
-  const int col4 = 4 * warp + cg;  // float4 column index of this thread (columns 4*col4 .. +3)
+  // float4 column index of this thread (columns 4*col4 .. +3)
+  const int col4 = 4 * warp + cg + (kD / 4 / kSplit) * (int)(blockIdx.x % kSplit);
   // staged window block: per token and row {alpha, k} and q; v; beta; q.k
   __shared__ float2 sak[kWB][kD];
   __shared__ float sq[kWB][kD], sv[kWB][kD], sb[kWB], sqk[kWB];
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   for (int t0 = 0; t0 < W; t0 += kWB) {
     const int nb = min(kWB, W - t0);
     if (t0 > 0) __syncthreads();  // every warp is done with the previous block
-    for (int e = tid; e < nb * kD; e += kWarps * 32) {
+    for (int e = tid; e < nb * kD; e += kW * 32) {
       const int u = e / kD, i = e % kD;
       const size_t in = ((size_t)bh * W + t0 + u) * kD + i;
       float gi = to_f(g[in]);
@@ -206,13 +215,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     }
     if (tid < nb) sb[tid] = to_f(beta[(size_t)bh * W + t0 + tid]);
     __syncthreads();
-    if (warp < nb) {  // q . k of token `warp`
+    for (int u = warp; u < nb; u += kW) {  // q . k of token u
       float acc = 0.f;
 #pragma unroll
-      for (int i = lane; i < kD; i += 32) acc += sq[warp][i] * sak[warp][i].y;
+      for (int i = lane; i < kD; i += 32) acc += sq[u][i] * sak[u][i].y;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) sqk[warp] = acc;
+      if (lane == 0) sqk[u] = acc;
     }
     __syncthreads();
     for (int u = 0; u < nb; ++u) {
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     if (kFused) {
       // Eq. 6 edge of the block's verified outputs: one warp per token, four columns per lane
       __syncthreads();
-      for (int u = warp; u < nb; u += kWarps) {
+      for (int u = warp; u < nb; u += kW) {
         const int t = t0 + u;
         if (t < nr) continue;
         const float4 ov = *reinterpret_cast<const float4 *>(&so[kFused ? u : 0][4 * lane]);
@@ -317,11 +326,11 @@ cudaError_t launch_dt(const SpecArgs &a, cudaStream_t st) {
   if (a.dk == kD && a.dv == kD) {
     const SpecEdges ed{a.A_log, a.g_min, a.gate, a.rms_w, a.eps};
     if (a.gate)
-      spec_replay_verify_d128_kernel<TIn, true><<<a.B * a.H, kWarps * 32, 0, st>>>(
+      spec_replay_verify_d128_kernel<TIn, true, 1><<<a.B * a.H, kWarps * 32, 0, st>>>(
           (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
           (TIn *)a.o, a.n_replay, a.H, a.W, a.scale, ed);
     else
-      spec_replay_verify_d128_kernel<TIn, false><<<a.B * a.H, kWarps * 32, 0, st>>>(
+      spec_replay_verify_d128_kernel<TIn, false, 2><<<a.B * a.H * 2, kWarps * 32 / 2, 0, st>>>(
           (const TIn *)a.q, (const TIn *)a.k, (const TIn *)a.v, (const TIn *)a.g, (const TIn *)a.beta, a.S,
           (TIn *)a.o, a.n_replay, a.H, a.W, a.scale, ed);
     return cudaGetLastError();
