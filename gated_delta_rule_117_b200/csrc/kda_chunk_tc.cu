@@ -37,12 +37,14 @@
 //   warps 0-3   chain:   thread e keeps column e of the fp32 state S in
 //                        registers (248 registers via setmaxnreg); per chunk
 //                        it writes S~^T, issues the [O | V~] MMAs, turns V~^T
-//                        into bf16 hi/lo operands, issues the dS/O MMAs,
-//                        applies the state update and stores the output tile;
+//                        into bf16 hi/lo operands, issues the dS/O MMAs and
+//                        applies the state update (with the fused Eq. 6 edge
+//                        it also normalises, gates and stores the output tile);
 //   warps 4-7   token A: TMA loads of q, k, g, the cumulative decay, the
 //                        rescaled operands and the Gram MMAs (chunk t + 2);
 //   warps 8-11  token B: A, L, the triangular solve, the U/W~ MMAs and -W~
-//                        (chunk t + 1).
+//                        (chunk t + 1), and the plain output tile of chunk
+//                        t - 2 (TMEM -> bf16 staging tile -> one TMA store).
 // One elected lane of a converged warp issues each MMA and TMA copy.  The issue
 // loops stay rolled: in isolation an unrolled loop issues a tcgen05.mma in ~20
 // cycles against ~70, but inside this pipeline the MMAs queue behind the other
