@@ -725,10 +725,16 @@ def pin_host(torch, t):
 
 
 def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
-    """Same metric through the C ABI from pinned host buffers: each step copies
-    the inputs host->device (into the device buffers the timed run used), runs
-    kda_chunk_fwd and copies o and h_T back to pinned host memory."""
-    stream = torch.cuda.current_stream()
+    """Same metric through the C ABI from pinned host buffers, for a stream of
+    steps: every step copies its inputs host->device, runs kda_chunk_fwd and
+    copies o and h_T back to pinned host memory, all inside the timed region.
+    Consecutive steps are pipelined as a serving loop would run them: two sets
+    of device buffers, uploads on one copy stream and downloads on another, so
+    step i+1's upload overlaps step i's compute and download (the host link is
+    full duplex); a step's compute waits for its own upload, and a buffer is
+    refilled only after the step two back has finished with it."""
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
     use_h0 = w.h0_std > 0
     names = ["q", "k", "v", "g", "beta"] + (["h0"] if use_h0 else [])
@@ -736,24 +742,44 @@ def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
     hx = {n: p[0] for n, p in pinned.items()}
     ho = torch.empty(B, H, T, dv, dtype=w.torch_dtype).pin_memory()
     hh = torch.empty(B, H, dk, dv, dtype=torch.float32).pin_memory()
-    do = torch.empty(B, H, T, dv, dtype=w.torch_dtype, device=dev)
-    dh = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    ins = [d, {n: torch.empty_like(d[n]) for n in names}]
+    outs = [(torch.empty(B, H, T, dv, dtype=w.torch_dtype, device=dev),
+             torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)) for _ in range(2)]
     ws = torch.empty(max(plan["workspace"], 16), dtype=torch.uint8, device=dev)
     dt = kda.KDA_DTYPE_BF16 if w.dtype == "bf16" else kda.KDA_DTYPE_F32
     h2d = sum(hx[n].numel() * hx[n].element_size() for n in names)
     d2h = ho.numel() * ho.element_size() + hh.numel() * hh.element_size()
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    count = [0]
 
     def step():
-        for n in names:
-            d[n].copy_(hx[n], non_blocking=True)
-        st = kda.kda_chunk_fwd(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["g"].data_ptr(),
-                               d["beta"].data_ptr(), d["h0"].data_ptr() if use_h0 else None, do.data_ptr(),
+        i = count[0]
+        count[0] += 1
+        b = i % 2
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(computed[b])  # step i - 2 has read these inputs
+            for n in names:
+                ins[b][n].copy_(hx[n], non_blocking=True)
+            uploaded[b].record(up)
+        comp.wait_event(uploaded[b])
+        if i >= 2:
+            comp.wait_event(downloaded[b])  # step i - 2's outputs have left
+        di, (do, dh) = ins[b], outs[b]
+        st = kda.kda_chunk_fwd(di["q"].data_ptr(), di["k"].data_ptr(), di["v"].data_ptr(), di["g"].data_ptr(),
+                               di["beta"].data_ptr(), di["h0"].data_ptr() if use_h0 else None, do.data_ptr(),
                                dh.data_ptr(), B, H, T, dk, dv, dt, args.chunk_size, 0.0, ws.data_ptr(), ws.numel(),
-                               stream.cuda_stream)
+                               comp.cuda_stream)
         if st != 0:
             raise kda.KdaError(st)
-        ho.copy_(do, non_blocking=True)
-        hh.copy_(dh, non_blocking=True)
+        computed[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            ho.copy_(do, non_blocking=True)
+            hh.copy_(dh, non_blocking=True)
+            downloaded[b].record(down)
 
     try:
         for _ in range(3):
@@ -761,14 +787,17 @@ def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        up.wait_event(a)  # the first timed upload starts inside the region
         for _ in range(args.steps):
             step()
-        b.record(stream)
+        for ev in downloaded:  # every step's download (hence its compute and upload) is done
+            comp.wait_event(ev)
+        e.record(comp)
         torch.cuda.synchronize()
         check_device_status(kda, "kda_chunk_fwd (e2e)")
-        ms = max_over_ranks(a.elapsed_time(b) / args.steps, dist, dev)
+        ms = max_over_ranks(a.elapsed_time(e) / args.steps, dist, dev)
     finally:
         for n, (t, reg) in pinned.items():
             if reg:
@@ -776,7 +805,8 @@ def measure_e2e(args, w, x, d, kda, torch, dev, plan, dist=None):
     world = dist.get_world_size() if dist is not None else 1
     return {"value": job_throughput(B * T, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "warmup": 3,
-            "host_buffers": "pinned (page-locked in place where possible)"}
+            "host_buffers": "pinned (page-locked in place where possible)",
+            "pipelining": "steps overlap: upload of step i+1 with compute and download of step i (two buffer sets)"}
 
 
 SPEC_WINDOW, SPEC_REPLAY = 4, 2  # window of 4 tokens: 2 accepted drafts replayed, bonus + 1 draft verified
