@@ -24,7 +24,9 @@ __device__ __forceinline__ float ld(const __nv_bfloat16 *p) { return __bfloat162
 __device__ __forceinline__ void st(float *p, float x) { *p = x; }
 __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 
-__device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
+// fast reciprocal division (the Eq. 6 gate of the fused paths uses the same form):
+// an IEEE division here made the pass instruction-bound
+__device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // Generic rows: any dv that is a multiple of 16 up to 128, either dtype.
 template <typename T>
