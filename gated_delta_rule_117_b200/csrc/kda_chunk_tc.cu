@@ -760,6 +760,8 @@ __global__ void __launch_bounds__(NT, 1)
           }
           float *part = reinterpret_cast<float *>(sm + kPart);
           part[warp * 32 + lane] = v[0];
+          // the previous chunk's output tile must be read out before this one is staged
+          if (warp == 0 && lane == 0 && t > 0) bulk_wait_read_all();
           named_sync(kBarChain, 128);
           if (warp == 0) {
             const float ssq = (part[lane] + part[32 + lane]) + (part[64 + lane] + part[96 + lane]);
@@ -788,7 +790,6 @@ __global__ void __launch_bounds__(NT, 1)
           tma_store_3d_warp(&mo, sm + kOst, 0, t0, bh);
           tma_store_3d_warp(&mo, sm + kOst + 4096, 64, t0, bh);
           bulk_commit_warp();
-          if (lane == 0) bulk_wait_read_all();  // the tile is rewritten next chunk
           if (kOut && has_next && *x.abort == 0) {  // every thread has read this chunk's gate tile
             mbar_arrive_expect_tx_warp(&x.bar[B_GATE], 2 * 4096);
             tma_load_3d_warp(sm + kGateT, &mgate, &x.bar[B_GATE], 0, t0 + C, bh);
@@ -942,7 +943,6 @@ __global__ void __launch_bounds__(NT, 1)
         tma_store_3d_warp(&mo, sm + kOst, 0, tb + t * C, bh);
         tma_store_3d_warp(&mo, sm + kOst + 4096, 64, tb + t * C, bh);
         bulk_commit_warp();
-        if (lane == 0) bulk_wait_read_all();  // the tile is rewritten only after token B's next named barrier
       }
     };
     int v_issued = -1;  // last chunk whose v copy was issued (abort path)
@@ -986,6 +986,8 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) Xa[r * 33 + j] = a[j];
       }
+      // the output tile staged at the top of this chunk is rewritten only after this barrier
+      if (out_b && t >= 2 && warp == 8 && lane == 0) bulk_wait_read_all();
       tc_fence_before();
       named_sync(kBarTokB, 128);
       if (!kTrans && quarter == 2) {
@@ -1055,8 +1057,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (out_b && nchunks > 0 && named_sync_and(kBarTokB, 128, *x.abort == 0)) {  // the last two output tiles
       if (nchunks >= 2) {
         out_plain(nchunks - 2);
-        // in the loop a named barrier of the chunk's own work always separates warp 8's
-        // wait for the staged tile to be read from the next tile's writes; here one is needed
+        if (warp == 8 && lane == 0) bulk_wait_read_all();  // before the last tile rewrites the staging
         named_sync(kBarTokB, 128);
       }
       out_plain(nchunks - 1);
