@@ -55,6 +55,28 @@ def test_plan(lib):
     assert kda.kda_chunk_fwd_workspace_size(1, 2, 64, 24, 16, 0, 0) == (1 << 64) - 1
 
 
+@pytest.mark.parametrize("B,H,T", [(1, 16, 4096), (1, 16, 1 << 20), (1, 8, 1024), (2, 2, 300), (1, 74, 512),
+                                   (8, 32, 8192), (1, 75, 1 << 16), (1, 1, 511), (3, 5, 2000)])
+def test_context_parallel_plan_and_workspace(lib, B, H, T):
+    # the tensor-core plan: P = min(148 // BH, T // 256) segments of whole 32-token chunks when
+    # BH <= 74 and P >= 2, else one CTA per chain; the workspace holds P - 1 transitions, P - 1
+    # states from zero and P entering states per chain (64 KiB fp32 each) and two 32-bit flags
+    # per transition, rounded up to 16 bytes
+    p = kda.kda_chunk_fwd_plan(B, H, T, 128, 128, kda.KDA_DTYPE_BF16, 0)
+    BH = B * H
+    P = min(148 // BH, T // 256) if BH <= 74 else 1
+    if P >= 2:
+        seg = -(-(-(-T // P)) // 32) * 32
+        P = -(-T // seg)
+        assert (p["segments"], p["segment_tokens"], p["launches"]) == (P, seg, 4)
+        flags = -(-(2 * BH * (P - 1) * 4) // 16) * 16
+        assert p["workspace"] == BH * (3 * P - 2) * 65536 + flags
+        assert (P - 1) * seg < T <= P * seg  # every segment holds tokens
+    else:
+        assert (p["segments"], p["segment_tokens"], p["launches"], p["workspace"]) == (1, T, 1, 0)
+    assert kda.kda_chunk_fwd_workspace_size(B, H, T, 128, 128, kda.KDA_DTYPE_BF16, 0) == p["workspace"]
+
+
 # Fake, never-dereferenced device addresses: validation must reject bad
 # arguments before any CUDA call.
 BASE = 1 << 40
