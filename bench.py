@@ -14,7 +14,9 @@ carries:
   * `parity` and `cpu_baseline`: the fp64 oracle over whole sampled chains of
     the main workload (run on host cores while the GPU legs run), compared
     with the timed run's own output, and its throughput;
-  * `e2e`: the same metric through the C ABI from pinned host buffers;
+  * `e2e`: the same metric through the C ABI from pinned host buffers, every
+    step's uploads and downloads inside the timed region, consecutive steps
+    pipelined over two copy streams and two device buffer sets;
   * secondary legs (checkpoints, output gate, fused gate, replay).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl libkda|reference]
